@@ -1,0 +1,194 @@
+/*
+ * haste.h -- C ABI of libhaste.so, a B200 (sm_100a) implementation of the HASTE
+ * group-shared fixed fan-in output layer for extreme multi-label classification.
+ *
+ * Source of the operations: "HASTE: Hardware-Aware Dynamic Sparse Training for
+ * Large Output Spaces" (summary page):
+ *   Methodology 1, Group-Shared Fixed Fan-In Sparsity
+ *     - structure: labels are partitioned into groups; all labels of a group share
+ *       one sparse set of input-feature indices (the fan-in pattern) and keep
+ *       independent weight vectors;
+ *     - hardware alignment: a group's input features are gathered into shared
+ *       memory once and reused by all labels of the group in a dense tensor-core
+ *       product;
+ *     - memory efficiency: indices are stored once per group.
+ *   Methodology 2, Head-Tail Decomposition: a dense classifier for the few frequent
+ *     (head) labels next to the sparse layer for the long tail.
+ *
+ * Notation: B batch rows, d input features, L tail labels in n_groups groups of G
+ * (group g owns labels [g*G, g*G+G)), k fan-in per group, H head labels.
+ *   idx [n_groups, k]  int32, each row strictly increasing in [0, d)
+ *   X   [B, d]   W [L, k] (W[l, s] multiplies feature idx[l / G, s])
+ *   logits, dY [B, L]   dW [L, k]   dX [B, d] (always fp32)
+ *   Xh  [B, d]   Wh [H, d]   logits_h, dY_h [B, H]   dWh [H, d]   dXh [B, d] fp32
+ * All matrices are contiguous and row-major.
+ *
+ * Conventions
+ *   - Tensor pointers are DEVICE pointers unless a parameter says "host".  The
+ *     caller owns every buffer it passes; the library owns only plan objects.
+ *   - Workspace is caller-provided; query its size first.  The library keeps no
+ *     pointer to it after the call's kernels finish.
+ *   - Every compute call is asynchronous on the given stream (a cudaStream_t cast
+ *     to void*, NULL = legacy default stream).  Argument errors are returned
+ *     synchronously before any launch; launch failures return HASTE_ERR_CUDA.
+ *     Nothing throws across the ABI.  haste_last_error() gives a message.
+ *   - Device-side bounded waits that run out set a device error word instead of
+ *     hanging; haste_device_status() synchronises and reports it.
+ *   - Supported by the GPU path: k*elem % 128 == 0 (k % 64 for bf16, k % 32 for
+ *     fp32), k <= 256, G % 16 == 0, 16 <= G <= 128, L*elem % 16 == 0, B <= 512;
+ *     head: H*elem and d*elem multiples of 16 bytes.
+ *     B <= 512.  Other shapes return HASTE_ERR_UNSUPPORTED_SHAPE.
+ *   - Results are deterministic: repeated calls give identical bits (fixed-order
+ *     reductions, no floating-point atomics).
+ */
+#ifndef HASTE_H
+#define HASTE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct haste_plan_s* haste_plan_t; /* opaque; owned by the library */
+typedef void* haste_stream_t;              /* a cudaStream_t */
+
+typedef enum {
+  HASTE_OK = 0,
+  HASTE_ERR_INVALID_ARG = 1,
+  HASTE_ERR_INDEX_UNSORTED_OR_DUP = 2,
+  HASTE_ERR_INDEX_OUT_OF_RANGE = 3,
+  HASTE_ERR_UNSUPPORTED_SHAPE = 4,
+  HASTE_ERR_WORKSPACE = 5,
+  HASTE_ERR_CUDA = 6,
+  HASTE_ERR_TIMEOUT = 7
+} haste_status_t;
+
+typedef enum { HASTE_F32 = 0, HASTE_BF16 = 1 } haste_dtype_t;
+
+/* Sparse positive labels per sample as a device CSR: row_ptr [B+1], ids [nnz],
+ * ids branch-local (tail: global id minus H; head: global id), each row sorted
+ * ascending without duplicates. */
+typedef struct {
+  const int32_t* row_ptr;
+  const int32_t* ids;
+} haste_targets_t;
+
+/* ABI version of this header (bumped on incompatible change). */
+int haste_abi_version(void);
+
+/* Thread-local message of the last failing call ("" when none). */
+const char* haste_last_error(void);
+
+/* Synchronise the stream and report the device error word: HASTE_OK, or
+ * HASTE_ERR_TIMEOUT if a kernel's bounded wait ran out (the word is then
+ * cleared), or HASTE_ERR_CUDA. */
+haste_status_t haste_device_status(haste_stream_t stream);
+
+/* Self-test of failure detection: launches a kernel whose bounded wait (20 ms)
+ * on a barrier that nothing releases runs out.  A following
+ * haste_device_status() returns HASTE_ERR_TIMEOUT once, and the context stays
+ * usable.  No GPU fault is involved. */
+haste_status_t haste_selftest_wait_timeout(haste_stream_t stream);
+
+/* Per-kernel timing without a profiler.  Between haste_profile_start() and
+ * haste_profile_stop(), every kernel the library launches is bracketed by CUDA
+ * events recorded on its launch stream.  haste_profile_stop() waits for those
+ * events, writes up to max_entries aggregates {kernel name, launches, summed
+ * milliseconds} (names are static strings) in order of first launch, turns
+ * recording off and returns the number of distinct kernels (-1 on a CUDA error). */
+typedef struct {
+  const char* name;
+  int32_t launches;
+  double total_ms;
+} haste_kernel_time_t;
+haste_status_t haste_profile_start(void);
+int32_t haste_profile_stop(haste_kernel_time_t* out, int32_t max_entries);
+
+/* ------------------------------------------------------------------ plan --- */
+
+/* Host-only core of the plan (no GPU needed): validates idx (host [n_groups*k])
+ * and writes the inverse map feature -> (group, slot) into host buffers:
+ * inv_off [d+1], inv_off[f] = number of entries whose feature is below f;
+ * inv_ent [n_groups*k], the entries e = g*k + s of feature f in ascending g.
+ * Validation: the first offending element in row-major order decides: out of
+ * [0, d) -> HASTE_ERR_INDEX_OUT_OF_RANGE; not above its predecessor in the row
+ * -> HASTE_ERR_INDEX_UNSORTED_OR_DUP.  Source: Methodology 1, structure (shared
+ * index set per group) and memory efficiency (indices stored once per group). */
+haste_status_t haste_plan_inverse_host(const int32_t* idx, int64_t n_groups, int32_t k, int32_t d,
+                                       int32_t* inv_off, int32_t* inv_ent);
+
+/* Build a plan: validate idx (host [n_groups*k]), build the inverse map, copy
+ * idx, inv_off and inv_ent to the current device (stream-ordered copies; the
+ * call returns after they complete).  *out receives the new plan. */
+haste_status_t haste_plan(haste_plan_t* out, const int32_t* idx, int64_t n_groups, int32_t G, int32_t k,
+                          int32_t d, haste_stream_t stream);
+
+/* Free a plan's device and host memory (synchronous).  NULL is accepted. */
+haste_status_t haste_plan_destroy(haste_plan_t plan);
+
+/* Index store of the plan: index_bytes = 4*n_groups*k (one int32 per group and
+ * slot, against 4*L*k for per-label fan-in); inverse_bytes = 4*(d+1+n_groups*k). */
+haste_status_t haste_plan_info(haste_plan_t plan, int64_t* index_bytes, int64_t* inverse_bytes);
+
+/* Copy the plan's DEVICE arrays back to host buffers (synchronous): idx
+ * [n_groups*k], inv_off [d+1], inv_ent [n_groups*k].  Any pointer may be NULL. */
+haste_status_t haste_plan_export(haste_plan_t plan, int32_t* idx, int32_t* inv_off, int32_t* inv_ent);
+
+/* Workspace bytes that every sparse-tail call below needs at batch B. */
+size_t haste_workspace_size(haste_plan_t plan, int32_t B, haste_dtype_t dtype);
+
+/* ------------------------------------------------------------- sparse tail --- */
+
+/* Forward: logits[b, g*G+j] = sum_s X[b, idx[g,s]] * W[g*G+j, s]  (fp32
+ * accumulation on the tensor cores; logits in the input dtype).
+ * Source: Methodology 1 (gather-once, dense tensor-core product per group). */
+haste_status_t haste_forward(haste_plan_t plan, int32_t B, haste_dtype_t dtype, const void* X, const void* W,
+                             void* logits, void* ws, size_t ws_bytes, haste_stream_t stream);
+
+/* dW[g*G+j, s] = sum_b dY[b, g*G+j] * X[b, idx[g,s]], dW in the input dtype. */
+haste_status_t haste_backward_dw(haste_plan_t plan, int32_t B, haste_dtype_t dtype, const void* X,
+                                 const void* dY, void* dW, void* ws, size_t ws_bytes, haste_stream_t stream);
+
+/* dX[b, f] (+)= sum over the (g, s) with idx[g,s] == f, in ascending g, of
+ * sum_j dY[b, g*G+j] * W[g*G+j, s]; fp32 output.  accumulate = 0 overwrites dX,
+ * 1 adds into it.  Features in no group receive exactly 0. */
+haste_status_t haste_backward_dx(haste_plan_t plan, int32_t B, haste_dtype_t dtype, const void* W,
+                                 const void* dY, float* dX, int accumulate, void* ws, size_t ws_bytes,
+                                 haste_stream_t stream);
+
+/* Fused tail training step (logits never reach global memory):
+ *   z = forward(X, W);  y[b,l] = 1 iff l is in tail_pos row b;
+ *   dY = grad_scale * (sigmoid(z) - y)   (rounded to the input dtype);
+ *   *loss = grad_scale * sum_{b,l} (softplus(z) - z*y)   (if loss != NULL, device fp32);
+ *   dW from dY as haste_backward_dw; dX (+)= from dY as haste_backward_dx.
+ * The loss is binary cross-entropy with logits summed over labels; grad_scale is
+ * normally 1/B.  (The page names no loss; BCE against sparse positives is this
+ * library's reading of the multi-label problem statement.) */
+haste_status_t haste_bce_step(haste_plan_t plan, int32_t B, haste_dtype_t dtype, const void* X, const void* W,
+                              haste_targets_t tail_pos, float grad_scale, float* loss, void* dW, float* dX,
+                              int accumulate, void* ws, size_t ws_bytes, haste_stream_t stream);
+
+/* -------------------------------------------------------------- dense head --- */
+
+/* Workspace bytes of the head calls at (B, H, d). */
+size_t haste_head_workspace_size(int32_t B, int32_t H, int32_t d, haste_dtype_t dtype);
+
+/* logits_h = Xh . Wh^T.  pos == NULL: logits_or_dY receives the logits.
+ * pos != NULL: it receives dY_h = grad_scale * (sigmoid(z) - y) and, if loss !=
+ * NULL, *loss = grad_scale * sum BCE (device fp32).  Source: Methodology 2. */
+haste_status_t haste_head_forward(int32_t B, int32_t H, int32_t d, haste_dtype_t dtype, const void* Xh,
+                                  const void* Wh, void* logits_or_dY, const haste_targets_t* pos, float grad_scale,
+                                  float* loss, void* ws, size_t ws_bytes, haste_stream_t stream);
+
+/* dWh = dY_h^T . Xh (input dtype) and dXh = dY_h . Wh (fp32). */
+haste_status_t haste_head_backward(int32_t B, int32_t H, int32_t d, haste_dtype_t dtype, const void* Xh,
+                                   const void* Wh, const void* dY_h, void* dWh, float* dXh, void* ws,
+                                   size_t ws_bytes, haste_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HASTE_H */

@@ -1,0 +1,651 @@
+// api.cu -- the C ABI of libhaste.so (declared in include/haste.h): plan builder,
+// argument checks, workspace layout and the launch sequences of the calls.
+//
+// The library is built as one translation unit (this file includes the kernel
+// sources) so that the device error word is a single static device variable.
+#include "../../include/haste.h"
+
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <thread>
+#include <vector>
+
+#include "head.cu"
+#include "tail.cu"
+
+using namespace haste;
+
+struct haste_plan_s {
+  int64_t n_groups;
+  int32_t G, k, d;
+  int device;
+  int32_t* idx_d;
+  int32_t* inv_off_d;
+  int32_t* inv_ent_d;
+};
+
+namespace {
+
+thread_local std::string g_err;
+
+haste_status_t fail(haste_status_t st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return st;
+}
+
+haste_status_t cuda_fail(cudaError_t e, const char* what) {
+  return fail(HASTE_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+#define HASTE_CUDA(call)                                       \
+  do {                                                         \
+    cudaError_t e_ = (call);                                   \
+    if (e_ != cudaSuccess) return cuda_fail(e_, #call);        \
+  } while (0)
+
+inline size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
+inline int elem_bytes(haste_dtype_t dt) { return dt == HASTE_F32 ? 4 : 2; }
+inline int round_up(int v, int m) { return (v + m - 1) / m * m; }
+
+struct DeviceInfo {
+  int sms = 0, smem_optin = 0, major = 0;
+};
+
+haste_status_t device_info(DeviceInfo& di) {
+  int dev = 0;
+  HASTE_CUDA(cudaGetDevice(&dev));
+  HASTE_CUDA(cudaDeviceGetAttribute(&di.sms, cudaDevAttrMultiProcessorCount, dev));
+  HASTE_CUDA(cudaDeviceGetAttribute(&di.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev));
+  HASTE_CUDA(cudaDeviceGetAttribute(&di.major, cudaDevAttrComputeCapabilityMajor, dev));
+  if (di.major != 10) return fail(HASTE_ERR_CUDA, "libhaste needs an sm_100 GPU (found compute capability %d.x)", di.major);
+  return HASTE_OK;
+}
+
+// Per-launch CUDA events on the launching stream while profiling is on
+// (haste_profile_start / haste_profile_stop).
+struct ProfRec {
+  const char* name;
+  cudaEvent_t a, b;
+};
+struct ProfState {
+  bool on = false;
+  std::vector<ProfRec> recs;
+  std::vector<cudaEvent_t> pool;
+  size_t next = 0;
+  std::mutex mu;
+};
+ProfState g_prof;
+
+cudaEvent_t prof_event() {
+  if (g_prof.next < g_prof.pool.size()) return g_prof.pool[g_prof.next++];
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+  g_prof.pool.push_back(e);
+  ++g_prof.next;
+  return e;
+}
+
+// Brackets one kernel launch with events when profiling is on.
+class ProfScope {
+ public:
+  ProfScope(const char* name, cudaStream_t s) : name_(name), s_(s) {
+    if (!g_prof.on) return;
+    std::lock_guard<std::mutex> g(g_prof.mu);
+    a_ = prof_event();
+    if (a_) cudaEventRecord(a_, s_);
+  }
+  ~ProfScope() {
+    if (!g_prof.on || !a_) return;
+    std::lock_guard<std::mutex> g(g_prof.mu);
+    cudaEvent_t b = prof_event();
+    if (!b) return;
+    cudaEventRecord(b, s_);
+    g_prof.recs.push_back({name_, a_, b});
+  }
+
+ private:
+  const char* name_;
+  cudaStream_t s_;
+  cudaEvent_t a_ = nullptr;
+};
+
+// Tiling of the dX pass: feature bands sized so the fp32 band accumulator fits
+// next to the W and dY tiles; group chunks so that all CTAs are resident.
+struct DxTiling {
+  int band, n_bands, n_chunks;
+};
+
+DxTiling dx_tiling(const haste_plan_s& p, int Bp, int elem, int sms, int smem_optin) {
+  DxTiling t{};
+  const size_t fixed = tail::smem_dx(elem, p.k, p.G, 0);
+  long avail = (long)smem_optin - (long)fixed;
+  int band = (int)std::min<long>(256, avail / 512);
+  band = std::max(8, band & ~7);
+  if (band > p.d) band = round_up(p.d, 8);
+  t.band = band;
+  t.n_bands = (p.d + band - 1) / band;
+  const int per_chunk = (Bp / 128) * t.n_bands;
+  int c = std::max(1, sms / per_chunk);
+  if ((int64_t)c > p.n_groups) c = (int)p.n_groups;
+  t.n_chunks = c;
+  return t;
+}
+
+// Workspace layout of the tail calls.
+struct TailWs {
+  size_t xt, dx_part, dy_buf, loss_part, total;
+};
+
+constexpr int kMaxLossParts = 4096;
+
+TailWs tail_ws(const haste_plan_s& p, int B, int elem, const DxTiling& t) {
+  TailWs w{};
+  const int Bp = round_up(B, 128);
+  size_t off = 0;
+  w.xt = off;
+  off = align256(off + (size_t)p.d * Bp * elem);
+  w.dx_part = off;
+  off = align256(off + (size_t)t.n_chunks * p.d * Bp * 4);
+  w.dy_buf = off;
+  off = align256(off + (size_t)B * p.n_groups * p.G * elem);
+  w.loss_part = off;
+  off = align256(off + (size_t)kMaxLossParts * 4);
+  w.total = off;
+  return w;
+}
+
+haste_status_t check_tail(const haste_plan_s* p, int B, haste_dtype_t dt, const DeviceInfo& di) {
+  if (!p) return fail(HASTE_ERR_INVALID_ARG, "plan is NULL");
+  if (dt != HASTE_F32 && dt != HASTE_BF16) return fail(HASTE_ERR_INVALID_ARG, "unknown dtype %d", (int)dt);
+  if (B <= 0) return fail(HASTE_ERR_INVALID_ARG, "B must be positive (got %d)", B);
+  const int E = elem_bytes(dt);
+  if ((p->k * E) % 128 || p->k > 256)
+    return fail(HASTE_ERR_UNSUPPORTED_SHAPE, "k=%d: the GPU path needs k*elem %% 128 == 0 and k <= 256", p->k);
+  if (p->G % 16 || p->G < 16 || p->G > 128)
+    return fail(HASTE_ERR_UNSUPPORTED_SHAPE, "G=%d: the GPU path needs G %% 16 == 0 and 16 <= G <= 128", p->G);
+  const int64_t L = p->n_groups * p->G;
+  if ((L * E) % 16) return fail(HASTE_ERR_UNSUPPORTED_SHAPE, "L*elem must be a multiple of 16 bytes");
+  if (B > 512) return fail(HASTE_ERR_UNSUPPORTED_SHAPE, "B=%d: the GPU path supports B <= 512", B);
+  const int Bp = round_up(B, 128);
+  const size_t need = std::max(std::max(tail::smem_forward(E, p->k, p->G), tail::smem_dw(E, p->k, p->G, Bp)),
+                               tail::smem_dx(E, p->k, p->G, 8));
+  if (need > (size_t)di.smem_optin)
+    return fail(HASTE_ERR_UNSUPPORTED_SHAPE, "tiles need %zu bytes of shared memory (> %d)", need, di.smem_optin);
+  return HASTE_OK;
+}
+
+haste_status_t check_ws(void* ws, size_t have, size_t need) {
+  if (have < need) return fail(HASTE_ERR_WORKSPACE, "workspace of %zu bytes is below the %zu needed", have, need);
+  if (need && !ws) return fail(HASTE_ERR_INVALID_ARG, "workspace pointer is NULL");
+  return HASTE_OK;
+}
+
+TailArgs make_args(const haste_plan_s& p, int B) {
+  TailArgs a{};
+  a.sh.B = B;
+  a.sh.Bp = round_up(B, 128);
+  a.sh.d = p.d;
+  a.sh.G = p.G;
+  a.sh.k = p.k;
+  a.sh.n_groups = p.n_groups;
+  a.sh.L = p.n_groups * p.G;
+  a.idx = p.idx_d;
+  return a;
+}
+
+template <typename T>
+cudaError_t xt(const TailArgs& a, const void* X, void* Xt, cudaStream_t st) {
+  return tail::launch_xt<T>(X, Xt, a.sh.B, a.sh.Bp, a.sh.d, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+int haste_abi_version(void) { return 1; }
+
+const char* haste_last_error(void) { return g_err.c_str(); }
+
+haste_status_t haste_device_status(haste_stream_t stream) {
+  HASTE_CUDA(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
+  int v = 0;
+  HASTE_CUDA(cudaMemcpyFromSymbol(&v, g_device_error, sizeof v));
+  if (v != 0) {
+    const int zero = 0;
+    HASTE_CUDA(cudaMemcpyToSymbol(g_device_error, &zero, sizeof zero));
+    return fail(HASTE_ERR_TIMEOUT, "a kernel's bounded wait ran out (device error word %d)", v);
+  }
+  return HASTE_OK;
+}
+
+haste_status_t haste_profile_start(void) {
+  std::lock_guard<std::mutex> g(g_prof.mu);
+  g_prof.recs.clear();
+  g_prof.next = 0;
+  g_prof.on = true;
+  return HASTE_OK;
+}
+
+int32_t haste_profile_stop(haste_kernel_time_t* out, int32_t max_entries) {
+  std::lock_guard<std::mutex> g(g_prof.mu);
+  g_prof.on = false;
+  std::vector<haste_kernel_time_t> agg;
+  for (const ProfRec& r : g_prof.recs) {
+    if (cudaEventSynchronize(r.b) != cudaSuccess) return -1;
+    float ms = 0.f;
+    if (cudaEventElapsedTime(&ms, r.a, r.b) != cudaSuccess) return -1;
+    auto it = std::find_if(agg.begin(), agg.end(), [&](const haste_kernel_time_t& k) { return !strcmp(k.name, r.name); });
+    if (it == agg.end()) {
+      agg.push_back({r.name, 1, (double)ms});
+    } else {
+      it->launches += 1;
+      it->total_ms += ms;
+    }
+  }
+  g_prof.recs.clear();
+  g_prof.next = 0;
+  const int32_t n = (int32_t)agg.size();
+  for (int32_t i = 0; out && i < n && i < max_entries; ++i) out[i] = agg[i];
+  return n;
+}
+
+haste_status_t haste_selftest_wait_timeout(haste_stream_t stream) {
+  DeviceInfo di;
+  haste_status_t st = device_info(di);
+  if (st != HASTE_OK) return st;
+  cudaError_t e = tail::launch_selftest_wait(20000000ull, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? HASTE_OK : cuda_fail(e, "haste_selftest_wait_timeout launch");
+}
+
+// Validation plus a stable counting sort of the entries by feature, split over
+// threads by contiguous group ranges: per-thread feature histograms, a prefix
+// over (feature, thread) in that order, then each thread scatters its own range.
+// Entries of one feature therefore land in ascending group order.
+haste_status_t haste_plan_inverse_host(const int32_t* idx, int64_t n_groups, int32_t k, int32_t d,
+                                       int32_t* inv_off, int32_t* inv_ent) {
+  if (!idx || !inv_off || !inv_ent) return fail(HASTE_ERR_INVALID_ARG, "NULL pointer");
+  if (n_groups <= 0 || k <= 0 || d <= 0) return fail(HASTE_ERR_INVALID_ARG, "n_groups, k and d must be positive");
+  if (n_groups * (int64_t)k > 0x7fffffffLL)
+    return fail(HASTE_ERR_UNSUPPORTED_SHAPE, "n_groups*k must fit in int32");
+  const int64_t n = n_groups * (int64_t)k;
+  unsigned hw = std::thread::hardware_concurrency();
+  int nt = (int)std::min<int64_t>(std::max(1u, std::min(hw, 32u)), std::max<int64_t>(1, n / (1 << 16)));
+  std::vector<int64_t> bounds(nt + 1);
+  for (int t = 0; t <= nt; ++t) bounds[t] = n_groups * t / nt;
+  std::vector<std::vector<int32_t>> hist(nt, std::vector<int32_t>(d, 0));
+  std::vector<int64_t> bad(nt, -1);  // first offending flat position per thread
+  std::vector<int> bad_code(nt, 0);
+
+  auto count = [&](int t) {
+    std::vector<int32_t>& h = hist[t];
+    for (int64_t g = bounds[t]; g < bounds[t + 1]; ++g) {
+      const int32_t* row = idx + g * k;
+      int32_t prev = -1;
+      for (int32_t s = 0; s < k; ++s) {
+        const int32_t f = row[s];
+        if ((uint32_t)f >= (uint32_t)d) {
+          bad[t] = g * k + s;
+          bad_code[t] = HASTE_ERR_INDEX_OUT_OF_RANGE;
+          return;
+        }
+        if (f <= prev) {
+          bad[t] = g * k + s;
+          bad_code[t] = HASTE_ERR_INDEX_UNSORTED_OR_DUP;
+          return;
+        }
+        prev = f;
+        ++h[f];
+      }
+    }
+  };
+  {
+    std::vector<std::thread> th;
+    for (int t = 1; t < nt; ++t) th.emplace_back(count, t);
+    count(0);
+    for (auto& x : th) x.join();
+  }
+  for (int t = 0; t < nt; ++t)
+    if (bad[t] >= 0)
+      return fail((haste_status_t)bad_code[t], "idx element %lld (group %lld, slot %lld) is %s",
+                  (long long)bad[t], (long long)(bad[t] / k), (long long)(bad[t] % k),
+                  bad_code[t] == HASTE_ERR_INDEX_OUT_OF_RANGE ? "out of [0, d)" : "not above its predecessor");
+  // prefix in (feature, thread) order: thread t's entries of feature f start at
+  // inv_off[f] + sum of the earlier threads' counts of f
+  int64_t run = 0;
+  for (int32_t f = 0; f < d; ++f) {
+    inv_off[f] = (int32_t)run;
+    for (int t = 0; t < nt; ++t) {
+      const int32_t c = hist[t][f];
+      hist[t][f] = (int32_t)run;
+      run += c;
+    }
+  }
+  inv_off[d] = (int32_t)run;
+  auto scatter = [&](int t) {
+    std::vector<int32_t>& pos = hist[t];
+    for (int64_t g = bounds[t]; g < bounds[t + 1]; ++g)
+      for (int32_t s = 0; s < k; ++s) inv_ent[pos[idx[g * k + s]]++] = (int32_t)(g * k + s);
+  };
+  {
+    std::vector<std::thread> th;
+    for (int t = 1; t < nt; ++t) th.emplace_back(scatter, t);
+    scatter(0);
+    for (auto& x : th) x.join();
+  }
+  return HASTE_OK;
+}
+
+haste_status_t haste_plan(haste_plan_t* out, const int32_t* idx, int64_t n_groups, int32_t G, int32_t k, int32_t d,
+                          haste_stream_t stream) {
+  if (!out) return fail(HASTE_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  if (G <= 0) return fail(HASTE_ERR_INVALID_ARG, "G must be positive");
+  if (n_groups * (int64_t)G > 0x7fffffffffffLL) return fail(HASTE_ERR_INVALID_ARG, "L too large");
+  const int64_t n = n_groups * (int64_t)k;
+  std::vector<int32_t> off((size_t)std::max(d, 0) + 1), ent((size_t)std::max<int64_t>(n, 0));
+  haste_status_t st = haste_plan_inverse_host(idx, n_groups, k, d, off.data(), ent.data());
+  if (st != HASTE_OK) return st;
+  haste_plan_s* p = new haste_plan_s{};
+  p->n_groups = n_groups;
+  p->G = G;
+  p->k = k;
+  p->d = d;
+  cudaGetDevice(&p->device);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMalloc(&p->idx_d, n * 4);
+  if (e == cudaSuccess) e = cudaMalloc(&p->inv_off_d, ((size_t)d + 1) * 4);
+  if (e == cudaSuccess) e = cudaMalloc(&p->inv_ent_d, n * 4);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(p->idx_d, idx, n * 4, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(p->inv_off_d, off.data(), ((size_t)d + 1) * 4, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(p->inv_ent_d, ent.data(), n * 4, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) {
+    haste_plan_destroy(p);
+    return cuda_fail(e, "plan upload");
+  }
+  *out = p;
+  return HASTE_OK;
+}
+
+haste_status_t haste_plan_destroy(haste_plan_t p) {
+  if (!p) return HASTE_OK;
+  cudaFree(p->idx_d);
+  cudaFree(p->inv_off_d);
+  cudaFree(p->inv_ent_d);
+  delete p;
+  return HASTE_OK;
+}
+
+haste_status_t haste_plan_info(haste_plan_t p, int64_t* index_bytes, int64_t* inverse_bytes) {
+  if (!p) return fail(HASTE_ERR_INVALID_ARG, "plan is NULL");
+  if (index_bytes) *index_bytes = 4 * p->n_groups * p->k;
+  if (inverse_bytes) *inverse_bytes = 4 * ((int64_t)p->d + 1 + p->n_groups * p->k);
+  return HASTE_OK;
+}
+
+haste_status_t haste_plan_export(haste_plan_t p, int32_t* idx, int32_t* inv_off, int32_t* inv_ent) {
+  if (!p) return fail(HASTE_ERR_INVALID_ARG, "plan is NULL");
+  const size_t n = (size_t)p->n_groups * p->k;
+  if (idx) HASTE_CUDA(cudaMemcpy(idx, p->idx_d, n * 4, cudaMemcpyDeviceToHost));
+  if (inv_off) HASTE_CUDA(cudaMemcpy(inv_off, p->inv_off_d, ((size_t)p->d + 1) * 4, cudaMemcpyDeviceToHost));
+  if (inv_ent) HASTE_CUDA(cudaMemcpy(inv_ent, p->inv_ent_d, n * 4, cudaMemcpyDeviceToHost));
+  return HASTE_OK;
+}
+
+size_t haste_workspace_size(haste_plan_t p, int32_t B, haste_dtype_t dt) {
+  if (!p || B <= 0) return 0;
+  DeviceInfo di;
+  if (device_info(di) != HASTE_OK) return 0;
+  const int Bp = round_up(B, 128);
+  const DxTiling t = dx_tiling(*p, Bp, elem_bytes(dt), di.sms, di.smem_optin);
+  return tail_ws(*p, B, elem_bytes(dt), t).total;
+}
+
+haste_status_t haste_forward(haste_plan_t p, int32_t B, haste_dtype_t dt, const void* X, const void* W,
+                             void* logits, void* ws, size_t ws_bytes, haste_stream_t stream) {
+  DeviceInfo di;
+  haste_status_t st = device_info(di);
+  if (st == HASTE_OK) st = check_tail(p, B, dt, di);
+  if (st != HASTE_OK) return st;
+  if (!X || !W || !logits) return fail(HASTE_ERR_INVALID_ARG, "NULL tensor pointer");
+  const int E = elem_bytes(dt);
+  const DxTiling t = dx_tiling(*p, round_up(B, 128), E, di.sms, di.smem_optin);
+  const TailWs w = tail_ws(*p, B, E, t);
+  if ((st = check_ws(ws, ws_bytes, w.total)) != HASTE_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  TailArgs a = make_args(*p, B);
+  a.Xt = static_cast<uint8_t*>(ws) + w.xt;
+  a.W = W;
+  a.logits = logits;
+  cudaError_t e;
+  {
+    ProfScope ps("xt", s);
+    e = dt == HASTE_BF16 ? xt<__nv_bfloat16>(a, X, const_cast<void*>(a.Xt), s)
+                         : xt<float>(a, X, const_cast<void*>(a.Xt), s);
+  }
+  if (e == cudaSuccess) {
+    ProfScope ps("tail_forward", s);
+    e = dt == HASTE_BF16 ? tail::launch_forward<__nv_bfloat16>(a, di.sms, s) : tail::launch_forward<float>(a, di.sms, s);
+  }
+  return e == cudaSuccess ? HASTE_OK : cuda_fail(e, "haste_forward launch");
+}
+
+haste_status_t haste_backward_dw(haste_plan_t p, int32_t B, haste_dtype_t dt, const void* X, const void* dY,
+                                 void* dW, void* ws, size_t ws_bytes, haste_stream_t stream) {
+  DeviceInfo di;
+  haste_status_t st = device_info(di);
+  if (st == HASTE_OK) st = check_tail(p, B, dt, di);
+  if (st != HASTE_OK) return st;
+  if (!X || !dY || !dW) return fail(HASTE_ERR_INVALID_ARG, "NULL tensor pointer");
+  const int E = elem_bytes(dt);
+  const DxTiling t = dx_tiling(*p, round_up(B, 128), E, di.sms, di.smem_optin);
+  const TailWs w = tail_ws(*p, B, E, t);
+  if ((st = check_ws(ws, ws_bytes, w.total)) != HASTE_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  TailArgs a = make_args(*p, B);
+  a.Xt = static_cast<uint8_t*>(ws) + w.xt;
+  a.dY = dY;
+  a.dW = dW;
+  cudaError_t e;
+  {
+    ProfScope ps("xt", s);
+    e = dt == HASTE_BF16 ? xt<__nv_bfloat16>(a, X, const_cast<void*>(a.Xt), s)
+                         : xt<float>(a, X, const_cast<void*>(a.Xt), s);
+  }
+  if (e == cudaSuccess) {
+    ProfScope ps("tail_dw", s);
+    e = dt == HASTE_BF16 ? tail::launch_backward_dw<__nv_bfloat16>(a, di.sms, s)
+                         : tail::launch_backward_dw<float>(a, di.sms, s);
+  }
+  return e == cudaSuccess ? HASTE_OK : cuda_fail(e, "haste_backward_dw launch");
+}
+
+haste_status_t haste_backward_dx(haste_plan_t p, int32_t B, haste_dtype_t dt, const void* W, const void* dY,
+                                 float* dX, int accumulate, void* ws, size_t ws_bytes, haste_stream_t stream) {
+  DeviceInfo di;
+  haste_status_t st = device_info(di);
+  if (st == HASTE_OK) st = check_tail(p, B, dt, di);
+  if (st != HASTE_OK) return st;
+  if (!W || !dY || !dX) return fail(HASTE_ERR_INVALID_ARG, "NULL tensor pointer");
+  const int E = elem_bytes(dt);
+  const DxTiling t = dx_tiling(*p, round_up(B, 128), E, di.sms, di.smem_optin);
+  const TailWs w = tail_ws(*p, B, E, t);
+  if ((st = check_ws(ws, ws_bytes, w.total)) != HASTE_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  TailArgs a = make_args(*p, B);
+  a.W = W;
+  a.dY = dY;
+  a.dX_part = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + w.dx_part);
+  a.band = t.band;
+  a.n_bands = t.n_bands;
+  a.n_chunks = t.n_chunks;
+  cudaError_t e;
+  {
+    ProfScope ps("tail_dx", s);
+    e = dt == HASTE_BF16 ? tail::launch_backward_dx<__nv_bfloat16>(a, false, s)
+                         : tail::launch_backward_dx<float>(a, false, s);
+  }
+  if (e == cudaSuccess) {
+    ProfScope ps("dx_reduce", s);
+    e = tail::launch_dx_reduce(a.dX_part, dX, t.n_chunks, p->d, a.sh.Bp, B, accumulate, s);
+  }
+  return e == cudaSuccess ? HASTE_OK : cuda_fail(e, "haste_backward_dx launch");
+}
+
+haste_status_t haste_bce_step(haste_plan_t p, int32_t B, haste_dtype_t dt, const void* X, const void* W,
+                              haste_targets_t pos, float grad_scale, float* loss, void* dW, float* dX,
+                              int accumulate, void* ws, size_t ws_bytes, haste_stream_t stream) {
+  DeviceInfo di;
+  haste_status_t st = device_info(di);
+  if (st == HASTE_OK) st = check_tail(p, B, dt, di);
+  if (st != HASTE_OK) return st;
+  if (!X || !W || !dW || !dX || !pos.row_ptr || !pos.ids) return fail(HASTE_ERR_INVALID_ARG, "NULL pointer");
+  const int E = elem_bytes(dt);
+  const int Bp = round_up(B, 128);
+  if ((Bp / 128) * p->G + (E == 4 ? (p->G + 31) / 32 * 32 : p->G) > 512)
+    return fail(HASTE_ERR_UNSUPPORTED_SHAPE, "(B/128 + 1) * G must fit the 512 TMEM columns");
+  if (tail::smem_step(E, p->k, p->G, Bp) > (size_t)di.smem_optin)
+    return fail(HASTE_ERR_UNSUPPORTED_SHAPE, "fused step tiles exceed shared memory");
+  const DxTiling t = dx_tiling(*p, Bp, E, di.sms, di.smem_optin);
+  const TailWs w = tail_ws(*p, B, E, t);
+  if ((st = check_ws(ws, ws_bytes, w.total)) != HASTE_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* wb = static_cast<uint8_t*>(ws);
+  TailArgs a = make_args(*p, B);
+  a.Xt = wb + w.xt;
+  a.W = W;
+  a.dW = dW;
+  a.dY_out = wb + w.dy_buf;
+  a.dX_part = reinterpret_cast<float*>(wb + w.dx_part);
+  a.loss_part = reinterpret_cast<float*>(wb + w.loss_part);
+  a.pos_ptr = pos.row_ptr;
+  a.pos_ids = pos.ids;
+  a.grad_scale = grad_scale;
+  a.band = t.band;
+  a.n_bands = t.n_bands;
+  a.n_chunks = t.n_chunks;
+  const int grid = dt == HASTE_BF16 ? tail::step_grid<__nv_bfloat16>(a, di.sms) : tail::step_grid<float>(a, di.sms);
+  if (grid <= 0 || grid > kMaxLossParts) return fail(HASTE_ERR_CUDA, "could not size the fused step grid");
+  cudaError_t e;
+  {
+    ProfScope ps("xt", s);
+    e = dt == HASTE_BF16 ? xt<__nv_bfloat16>(a, X, const_cast<void*>(a.Xt), s)
+                         : xt<float>(a, X, const_cast<void*>(a.Xt), s);
+  }
+  if (e == cudaSuccess) {
+    ProfScope ps("tail_step", s);
+    e = dt == HASTE_BF16 ? tail::launch_step<__nv_bfloat16>(a, grid, s) : tail::launch_step<float>(a, grid, s);
+  }
+  if (e == cudaSuccess) {
+    ProfScope ps("tail_dx", s);
+    e = dt == HASTE_BF16 ? tail::launch_backward_dx<__nv_bfloat16>(a, true, s)
+                         : tail::launch_backward_dx<float>(a, true, s);
+  }
+  if (e == cudaSuccess) {
+    ProfScope ps("dx_reduce", s);
+    e = tail::launch_dx_reduce(a.dX_part, dX, t.n_chunks, p->d, Bp, B, accumulate, s);
+  }
+  if (e == cudaSuccess && loss) {
+    ProfScope ps("loss_reduce", s);
+    e = tail::launch_loss_reduce(a.loss_part, grid, grad_scale, loss, s);
+  }
+  return e == cudaSuccess ? HASTE_OK : cuda_fail(e, "haste_bce_step launch");
+}
+
+// ------------------------------------------------------------------- head
+namespace {
+struct HeadWs {
+  size_t loss_part, dxh_part, total;
+};
+HeadWs head_ws(int B, int H, int d, int E) {
+  HeadWs w{};
+  size_t off = 0;
+  w.loss_part = off;
+  off = align256(off + (size_t)head::fwd_tiles(B, H) * 4);
+  w.dxh_part = off;
+  const int S = head::dxh_splits(H, E);
+  off = align256(off + (S > 1 ? (size_t)S * B * d * 4 : 0));
+  w.total = off;
+  return w;
+}
+haste_status_t check_head(int B, int H, int d, haste_dtype_t dt) {
+  if (dt != HASTE_F32 && dt != HASTE_BF16) return fail(HASTE_ERR_INVALID_ARG, "unknown dtype %d", (int)dt);
+  if (B <= 0 || H <= 0 || d <= 0) return fail(HASTE_ERR_INVALID_ARG, "B, H and d must be positive");
+  const int E = elem_bytes(dt);
+  if ((d * E) % 16 || (H * E) % 16)
+    return fail(HASTE_ERR_UNSUPPORTED_SHAPE, "H and d must be multiples of %d", 16 / E);
+  return HASTE_OK;
+}
+}  // namespace
+
+size_t haste_head_workspace_size(int32_t B, int32_t H, int32_t d, haste_dtype_t dt) {
+  if (B <= 0 || H <= 0 || d <= 0) return 0;
+  return head_ws(B, H, d, elem_bytes(dt)).total;
+}
+
+haste_status_t haste_head_forward(int32_t B, int32_t H, int32_t d, haste_dtype_t dt, const void* Xh, const void* Wh,
+                                  void* out, const haste_targets_t* pos, float grad_scale, float* loss, void* ws,
+                                  size_t ws_bytes, haste_stream_t stream) {
+  DeviceInfo di;
+  haste_status_t st = device_info(di);
+  if (st == HASTE_OK) st = check_head(B, H, d, dt);
+  if (st != HASTE_OK) return st;
+  if (!Xh || !Wh || !out) return fail(HASTE_ERR_INVALID_ARG, "NULL tensor pointer");
+  if (pos && (!pos->row_ptr || !pos->ids)) return fail(HASTE_ERR_INVALID_ARG, "NULL targets");
+  const HeadWs w = head_ws(B, H, d, elem_bytes(dt));
+  if ((st = check_ws(ws, ws_bytes, w.total)) != HASTE_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  float* lp = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + w.loss_part);
+  const int32_t* rp = pos ? pos->row_ptr : nullptr;
+  const int32_t* ids = pos ? pos->ids : nullptr;
+  cudaError_t e;
+  {
+    ProfScope ps("head_forward", s);
+    e = dt == HASTE_BF16 ? head::forward<__nv_bfloat16>(B, H, d, Xh, Wh, out, rp, ids, grad_scale, lp, s)
+                         : head::forward<float>(B, H, d, Xh, Wh, out, rp, ids, grad_scale, lp, s);
+  }
+  if (e == cudaSuccess && pos && loss) {
+    ProfScope ps("loss_reduce", s);
+    e = tail::launch_loss_reduce(lp, head::fwd_tiles(B, H), grad_scale, loss, s);
+  }
+  return e == cudaSuccess ? HASTE_OK : cuda_fail(e, "haste_head_forward launch");
+}
+
+haste_status_t haste_head_backward(int32_t B, int32_t H, int32_t d, haste_dtype_t dt, const void* Xh, const void* Wh,
+                                   const void* dYh, void* dWh, float* dXh, void* ws, size_t ws_bytes,
+                                   haste_stream_t stream) {
+  DeviceInfo di;
+  haste_status_t st = device_info(di);
+  if (st == HASTE_OK) st = check_head(B, H, d, dt);
+  if (st != HASTE_OK) return st;
+  if (!Xh || !Wh || !dYh || !dWh || !dXh) return fail(HASTE_ERR_INVALID_ARG, "NULL tensor pointer");
+  const HeadWs w = head_ws(B, H, d, elem_bytes(dt));
+  if ((st = check_ws(ws, ws_bytes, w.total)) != HASTE_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  float* part = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + w.dxh_part);
+  cudaError_t e;
+  {
+    ProfScope ps("head_dw", s);
+    e = dt == HASTE_BF16 ? head::backward_dw<__nv_bfloat16>(B, H, d, Xh, dYh, dWh, s)
+                         : head::backward_dw<float>(B, H, d, Xh, dYh, dWh, s);
+  }
+  if (e == cudaSuccess) {
+    ProfScope ps("head_dx", s);
+    e = dt == HASTE_BF16 ? head::backward_dx<__nv_bfloat16>(B, H, d, Wh, dYh, dXh, part, s)
+                         : head::backward_dx<float>(B, H, d, Wh, dYh, dXh, part, s);
+  }
+  return e == cudaSuccess ? HASTE_OK : cuda_fail(e, "haste_head_backward launch");
+}
+
+}  // extern "C"

@@ -1,0 +1,318 @@
+// head.cu -- the dense head classifier on the 5th-gen tensor cores.
+//
+// HASTE ("Hardware-Aware Dynamic Sparse Training for Large Output Spaces"),
+// Methodology 2 "Head-Tail Decomposition": the few frequent labels are modelled by
+// a standard dense classifier next to the group-shared sparse tail.
+//   forward : logits_h = Xh . Wh^T               (M = batch, N = H, K = d)
+//   dWh     : dWh = dY_h^T . Xh                   (M = H, N = d, K = batch)
+//   dXh     : dXh = dY_h . Wh                     (M = batch, N = d, K = H)
+// One tcgen05 GEMM kernel D[M,N] = A[M,K] . B[N,K]^T covers the three products;
+// each operand is read from global memory either K-contiguous or MN-contiguous
+// and staged into the matching 128B-swizzled canonical layout.
+#include "common.cuh"
+
+namespace haste {
+namespace {
+
+constexpr int kGThreads = 128;
+constexpr int kBM = 128, kBN = 128;
+
+enum Epi : int { kEpiStore = 0, kEpiStoreF32 = 1, kEpiPartial = 2, kEpiBce = 3 };
+
+struct GemmArgs {
+  const void* A;   // element (m, k) at A[m*lda + k] (K-major) or A[k*lda + m] (MN-major)
+  const void* Bm;  // element (n, k) at B[n*ldb + k] (K-major) or B[k*ldb + n] (MN-major)
+  int64_t lda, ldb;
+  int M, N, K;
+  int k_per_split;
+  void* C;          // output [M, N] row-major (ldc), or partials [splits, M, N] fp32
+  int64_t ldc;
+  // BCE epilogue
+  const int32_t* pos_ptr;
+  const int32_t* pos_ids;
+  float scale;
+  float* loss_part;
+};
+
+// Stage a 128 x BK tile of an operand whose rows are the M (or N) index.
+template <typename T, bool kMN>
+__device__ __forceinline__ void load_operand(uint32_t s, const T* __restrict__ p, int64_t ld, int rows, int K,
+                                             int r0, int k0, int BK) {
+  constexpr int CW = 16 / sizeof(T);
+  if constexpr (!kMN) {
+    // K-major: [k-block][row][128B]
+    const int cpr = BK / CW;
+    for (int i = threadIdx.x; i < 128 * cpr; i += blockDim.x) {
+      const int r = i / cpr, cc = i % cpr;
+      const int gr = r0 + r, gk = k0 + cc * CW;
+      const bool in = gr < rows && gk < K;
+      const T* src = in ? p + (int64_t)gr * ld + gk : p;
+      const uint32_t off = (uint32_t)((cc >> 3) * 128 * 128 + r * 128 + (cc & 7) * 16);
+      cp_async16(s + sw128(off), src, in ? 16u : 0u);
+    }
+  } else {
+    // MN-major: [row-block of R][k][128B]
+    const int cpr = 128 / CW;
+    for (int i = threadIdx.x; i < BK * cpr; i += blockDim.x) {
+      const int kr = i / cpr, cc = i % cpr;
+      const int gk = k0 + kr, gr = r0 + cc * CW;
+      const bool in = gk < K && gr < rows;
+      const T* src = in ? p + (int64_t)gk * ld + gr : p;
+      const uint32_t off = (uint32_t)((cc >> 3) * BK * 128 + kr * 128 + (cc & 7) * 16);
+      cp_async16(s + swz<T, true>(off), src, in ? 16u : 0u);
+    }
+  }
+}
+
+template <typename T, bool kMN>
+__device__ __forceinline__ uint64_t operand_desc(uint32_t s, int kk, int BK) {
+  constexpr int R = 128 / sizeof(T), KI = Elem<T>::kMmaK;
+  if constexpr (!kMN) {
+    return make_sdesc(s + (uint32_t)(((kk * KI) / R) * 128 * 128 + (kk % (R / KI)) * 32), 16, 1024, kLayoutSw128);
+  } else {
+    return mn_desc<T>(s + (uint32_t)(kk * KI * 128), (uint32_t)BK * 128);
+  }
+}
+
+template <typename T, bool kAMN, bool kBMN, int kEpi>
+__global__ void __launch_bounds__(kGThreads, 1) k_gemm(GemmArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  constexpr int R = 128 / sizeof(T), KI = Elem<T>::kMmaK;
+  constexpr int BK = 2 * R;  // two 128B rows of K per stage
+  const uint32_t base = align1024(smem_u32(smem));
+  const uint32_t sa = base;
+  const uint32_t sb = sa + (uint32_t)kBM * BK * sizeof(T);
+  uint8_t* gen = smem + (sb + (uint32_t)kBN * BK * sizeof(T) - smem_u32(smem));
+  uint64_t* bar = reinterpret_cast<uint64_t*>(gen);
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bar + 1);
+  int* abort_flag = reinterpret_cast<int*>(tslot + 1);
+  float* red = reinterpret_cast<float*>(abort_flag + 1);
+
+  const int m0 = blockIdx.x * kBM, n0 = blockIdx.y * kBN, split = blockIdx.z;
+  const int k_begin = split * a.k_per_split;
+  const int k_end = min(a.K, k_begin + a.k_per_split);
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (threadIdx.x < 32) {
+    tmem_alloc(tslot, 128);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tslot;
+  uint32_t phase = 0;
+  const uint32_t idesc = make_idesc(Elem<T>::kFmt, kAMN ? 1u : 0u, kBMN ? 1u : 0u, 128, kBN);
+  const T* A = static_cast<const T*>(a.A);
+  const T* Bm = static_cast<const T*>(a.Bm);
+  bool ok = true;
+
+  for (int k0 = k_begin; k0 < k_end; k0 += BK) {
+    load_operand<T, kAMN>(sa, A, a.lda, a.M, k_end, m0, k0, BK);
+    load_operand<T, kBMN>(sb, Bm, a.ldb, a.N, k_end, n0, k0, BK);
+    cp_async_commit();
+    cp_async_wait_all();
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      tc_fence_after();
+      for (int kk = 0; kk < BK / KI; ++kk)
+        mma_ss<Elem<T>::kTF32>(tmem, operand_desc<T, kAMN>(sa, kk, BK), operand_desc<T, kBMN>(sb, kk, BK), idesc,
+                               (k0 > k_begin || kk > 0) ? 1u : 0u);
+      mma_commit(bar);
+    }
+    const bool w = mbar_wait(bar, phase);
+    phase ^= 1u;
+    if (!w) *abort_flag = 1;
+    tc_fence_after();
+    __syncthreads();
+    if (*abort_flag) {
+      ok = false;
+      break;
+    }
+  }
+
+  const int m = m0 + threadIdx.x;
+  const uint32_t lane = tmem + (((threadIdx.x / 32) * 32u) << 16);
+  float loss_acc = 0.f;
+  if (ok && k_end > k_begin) {
+    uint64_t ym0 = 0, ym1 = 0;
+    if constexpr (kEpi == kEpiBce) {
+      if (m < a.M)
+        for (int p = a.pos_ptr[m]; p < a.pos_ptr[m + 1]; ++p) {
+          const int l = a.pos_ids[p] - n0;
+          if (l >= 0 && l < 64) ym0 |= 1ull << l;
+          else if (l >= 64 && l < 128) ym1 |= 1ull << (l - 64);
+        }
+    }
+    for (int c = 0; c < kBN; c += 16) {
+      float v[16];
+      tmem_ld16(lane + (uint32_t)c, v);
+      tmem_wait_ld();
+      if (m >= a.M) continue;
+      const int n = n0 + c;
+      if constexpr (kEpi == kEpiPartial) {
+        float* dst = static_cast<float*>(a.C) + ((int64_t)split * a.M + m) * a.N + n;
+        for (int i = 0; i < 16; ++i)
+          if (n + i < a.N) dst[i] = v[i];
+      } else if constexpr (kEpi == kEpiStoreF32) {
+        float* dst = static_cast<float*>(a.C) + (int64_t)m * a.ldc + n;
+        for (int i = 0; i < 16; ++i)
+          if (n + i < a.N) dst[i] = v[i];
+      } else {
+        if constexpr (kEpi == kEpiBce) {
+          float lin = 0.f, prod = 1.f;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int j = c + i;
+            const uint64_t mk = j < 64 ? ym0 : ym1;
+            const float y = ((mk >> (j & 63)) & 1ull) ? 1.f : 0.f;
+            const float th = tanh_approx(0.5f * v[i]);
+            const bool in = n + i < a.N;
+            lin += in ? fmaxf(v[i], 0.f) - v[i] * y : 0.f;
+            prod *= in ? fmaf(0.5f, fabsf(th), 0.5f) : 1.f;
+            v[i] = a.scale * (fmaf(0.5f, th, 0.5f) - y);
+          }
+          loss_acc += lin - __logf(prod);
+        }
+        T* dst = static_cast<T*>(a.C) + (int64_t)m * a.ldc + n;
+        for (int i = 0; i < 16; ++i)
+          if (n + i < a.N) dst[i] = Elem<T>::from_f(v[i]);
+      }
+    }
+  }
+  if constexpr (kEpi == kEpiBce) {
+    float v = loss_acc;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+    __syncthreads();
+    if (threadIdx.x == 0) a.loss_part[blockIdx.y * gridDim.x + blockIdx.x] = ((red[0] + red[1]) + red[2]) + red[3];
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
+  }
+}
+
+// out[m, n] = sum over splits s ascending of P[s, m, n]
+__global__ void k_split_reduce(const float* __restrict__ P, float* __restrict__ out, int S, int64_t MN) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < MN; i += (int64_t)gridDim.x * blockDim.x) {
+    float s = 0.f;
+    for (int sp = 0; sp < S; ++sp) s += P[sp * MN + i];
+    out[i] = s;
+  }
+}
+
+template <typename T, bool kAMN, bool kBMN, int kEpi>
+cudaError_t run_gemm(const GemmArgs& a, int splits, cudaStream_t st) {
+  constexpr int BK = 2 * (128 / (int)sizeof(T));
+  const size_t smem = 1024 + (size_t)(kBM + kBN) * BK * sizeof(T) + 64;
+  auto kern = k_gemm<T, kAMN, kBMN, kEpi>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((a.M + kBM - 1) / kBM, (a.N + kBN - 1) / kBN, splits);
+  kern<<<grid, kGThreads, smem, st>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+namespace head {
+
+// Work split of dXh (K = H can be long): K chunks of a multiple of the stage depth.
+int dxh_splits(int H, int elem) {
+  const int BK = 2 * (128 / elem);
+  int s = H / 1024;
+  if (s < 1) s = 1;
+  if (s > 32) s = 32;
+  while (s > 1 && ((H + s - 1) / s) % BK) --s;
+  return s;
+}
+
+int fwd_tiles(int B, int H) { return ((B + kBM - 1) / kBM) * ((H + kBN - 1) / kBN); }
+
+template <typename T>
+cudaError_t forward(int B, int H, int d, const void* Xh, const void* Wh, void* out, const int32_t* pos_ptr,
+                    const int32_t* pos_ids, float scale, float* loss_part, cudaStream_t st) {
+  GemmArgs a{};
+  a.A = Xh;
+  a.lda = d;
+  a.Bm = Wh;
+  a.ldb = d;
+  a.M = B;
+  a.N = H;
+  a.K = d;
+  a.k_per_split = d;
+  a.C = out;
+  a.ldc = H;
+  if (pos_ptr) {
+    a.pos_ptr = pos_ptr;
+    a.pos_ids = pos_ids;
+    a.scale = scale;
+    a.loss_part = loss_part;
+    return run_gemm<T, false, false, kEpiBce>(a, 1, st);
+  }
+  return run_gemm<T, false, false, kEpiStore>(a, 1, st);
+}
+
+// dWh = dY_h^T . Xh : A(m=h, k=b) = dY_h[b, h] (MN-major), B(n=f, k=b) = Xh[b, f] (MN-major)
+template <typename T>
+cudaError_t backward_dw(int B, int H, int d, const void* Xh, const void* dYh, void* dWh, cudaStream_t st) {
+  GemmArgs a{};
+  a.A = dYh;
+  a.lda = H;
+  a.Bm = Xh;
+  a.ldb = d;
+  a.M = H;
+  a.N = d;
+  a.K = B;
+  a.k_per_split = B;
+  a.C = dWh;
+  a.ldc = d;
+  return run_gemm<T, true, true, kEpiStore>(a, 1, st);
+}
+
+// dXh = dY_h . Wh : A(m=b, k=h) = dY_h[b, h] (K-major), B(n=f, k=h) = Wh[h, f] (MN-major);
+// split over K = H into fp32 partials reduced in a fixed order.
+template <typename T>
+cudaError_t backward_dx(int B, int H, int d, const void* Wh, const void* dYh, float* dXh, float* part,
+                        cudaStream_t st) {
+  const int S = dxh_splits(H, sizeof(T));
+  GemmArgs a{};
+  a.A = dYh;
+  a.lda = H;
+  a.Bm = Wh;
+  a.ldb = d;
+  a.M = B;
+  a.N = d;
+  a.K = H;
+  a.k_per_split = (H + S - 1) / S;
+  a.C = S > 1 ? (void*)part : (void*)dXh;
+  a.ldc = d;
+  if (S == 1) return run_gemm<T, false, true, kEpiStoreF32>(a, 1, st);
+  cudaError_t e = run_gemm<T, false, true, kEpiPartial>(a, S, st);
+  if (e != cudaSuccess) return e;
+  const int64_t MN = (int64_t)B * d;
+  k_split_reduce<<<(int)((MN + 255) / 256 < 1184 ? (MN + 255) / 256 : 1184), 256, 0, st>>>(part, dXh, S, MN);
+  return cudaGetLastError();
+}
+
+template cudaError_t forward<float>(int, int, int, const void*, const void*, void*, const int32_t*, const int32_t*,
+                                    float, float*, cudaStream_t);
+template cudaError_t forward<__nv_bfloat16>(int, int, int, const void*, const void*, void*, const int32_t*,
+                                            const int32_t*, float, float*, cudaStream_t);
+template cudaError_t backward_dw<float>(int, int, int, const void*, const void*, void*, cudaStream_t);
+template cudaError_t backward_dw<__nv_bfloat16>(int, int, int, const void*, const void*, void*, cudaStream_t);
+template cudaError_t backward_dx<float>(int, int, int, const void*, const void*, float*, float*, cudaStream_t);
+template cudaError_t backward_dx<__nv_bfloat16>(int, int, int, const void*, const void*, float*, float*,
+                                                cudaStream_t);
+
+}  // namespace head
+}  // namespace haste

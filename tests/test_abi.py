@@ -1,0 +1,70 @@
+"""The C ABI without a GPU: the library loads, exports every function that
+include/haste.h declares, and its host plan builder is bit-exact against the
+oracle's independent inverse-map construction (HASTE summary page,
+Methodology 1: one fan-in index set per group, stored once per group)."""
+import os
+import re
+
+import numpy as np
+import pytest
+
+from oracle import oracle as O
+from structured_sparse_output_b200 import haste as H
+from structured_sparse_output_b200 import inputs as I
+
+
+def _declared():
+    text = open(H.HEADER_PATH).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(haste_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    names = _declared()
+    assert len(names) >= 16
+    lib = H.lib()
+    missing = [n for n in names if not hasattr(lib, n)]
+    assert not missing, missing
+    assert lib.haste_abi_version() == 1
+
+
+@pytest.mark.parametrize("n_groups,k,d", [(256, 32, 256), (20_944, 128, 768), (1000, 64, 97), (3, 5, 5)])
+def test_host_plan_bit_exact_vs_oracle(n_groups, k, d):
+    idx = I.make_idx(n_groups, k, d, 7)
+    off, ent = H.haste_plan_inverse_host(idx, d)
+    st, ref_off, ref_ent = O.plan(idx, d)
+    assert st == O.OK
+    assert np.array_equal(off, ref_off) and np.array_equal(ent, ref_ent)
+
+
+def test_host_plan_error_codes_match_oracle():
+    cases = [
+        (np.array([[0, 4], [1, 2]], dtype=np.int32), 4),
+        (np.array([[2, 2]], dtype=np.int32), 4),
+        (np.array([[3, 1], [0, 9]], dtype=np.int32), 4),
+        (np.array([[0, 9], [3, 1]], dtype=np.int32), 4),
+        (np.array([[-5, 1]], dtype=np.int32), 4),
+    ]
+    big = I.make_idx(5000, 16, 64, 1)
+    big[4321, 7] = big[4321, 6]          # a duplicate deep inside, on another thread's range
+    cases.append((big, 64))
+    for idx, d in cases:
+        ref = O.validate(idx, d)
+        assert ref != O.OK
+        with pytest.raises(H.HasteError) as ei:
+            H.haste_plan_inverse_host(idx, d)
+        assert ei.value.status == ref
+
+
+def test_head_workspace_size_is_host_only():
+    assert H.haste_head_workspace_size(256, 4096, 768, H.HASTE_BF16) > 0
+    assert H.haste_head_workspace_size(0, 4096, 768, H.HASTE_BF16) == 0
+
+
+def test_calls_fail_cleanly_without_gpu():
+    torch = pytest.importorskip("torch")
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    st = H.lib().haste_head_forward(256, 256, 256, H.HASTE_BF16, None, None, None, None, 1.0, None, None, 0, None)
+    assert st == H.HASTE_ERR_CUDA
+    assert H.lib().haste_last_error()

@@ -1,0 +1,235 @@
+"""GPU parity of the C-ABI path against the fp64 oracle (B200, sm_100a).
+
+Every call goes through libhaste.so; inputs come from the seeded generator and are
+fed to both sides bit-identically.  Floating-point tolerance: relative L2 <= 5e-3
+and elementwise max-abs relative error <= 2e-2 (helpers.assert_close); the plan
+is bit-exact.  Shapes span several tiles with ragged tails (batch not a multiple
+of 128, feature bands cut short, group counts not a multiple of the grid).
+Source: "HASTE: Hardware-Aware Dynamic Sparse Training for Large Output Spaces"
+(summary page), Methodology 1 and 2.
+"""
+import math
+
+import numpy as np
+import pytest
+
+from oracle import oracle as O
+from structured_sparse_output_b200 import haste as H
+from structured_sparse_output_b200 import inputs as I
+from tests.helpers import assert_close, to_np64, to_torch
+
+pytestmark = pytest.mark.gpu
+torch = pytest.importorskip("torch")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _need_gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    H.lib()
+    yield
+    torch.cuda.synchronize()
+    assert H.haste_device_status() == H.HASTE_OK
+
+
+def _inputs(B, d, n_groups, G, k, dtype, seed=0):
+    idx = I.make_idx(n_groups, k, d, seed)
+    X = I.make_normal((B, d), 1.0, seed, 1, dtype)
+    W = I.make_normal((n_groups * G, k), 1.0 / math.sqrt(k), seed, 2, dtype)
+    dY = I.make_normal((B, n_groups * G), 1.0, seed, 3, dtype)
+    return idx, X, W, dY
+
+
+def _ws(plan, B, dtype_code):
+    n = plan.workspace_size(B, dtype_code)
+    assert n > 0
+    return torch.empty(n, dtype=torch.uint8, device="cuda")
+
+
+TAIL_CASES = [
+    dict(B=32, d=256, n_groups=256, G=16, k=32, dtype="f32"),       # the tiny workload
+    dict(B=130, d=200, n_groups=100, G=32, k=64, dtype="f32"),
+    dict(B=200, d=320, n_groups=333, G=32, k=64, dtype="bf16"),
+    dict(B=256, d=768, n_groups=500, G=64, k=128, dtype="bf16"),
+    dict(B=512, d=1024, n_groups=256, G=16, k=128, dtype="bf16"),
+    dict(B=128, d=512, n_groups=64, G=128, k=64, dtype="bf16"),
+    dict(B=64, d=96, n_groups=40, G=48, k=64, dtype="bf16"),
+]
+
+
+def _case_id(c):
+    return "B{B}_d{d}_n{n_groups}_G{G}_k{k}_{dtype}".format(**c)
+
+
+@pytest.mark.parametrize("case", TAIL_CASES, ids=_case_id)
+def test_tail_forward_dw_dx(case):
+    B, d, n_groups, G, k, dt = (case[x] for x in ("B", "d", "n_groups", "G", "k", "dtype"))
+    idx, X, W, dY = _inputs(B, d, n_groups, G, k, dt)
+    plan = H.haste_plan(idx, G, d)
+    Xt, Wt, dYt = to_torch(X), to_torch(W), to_torch(dY)
+    code = H.dtype_code(Xt)
+    ws = _ws(plan, B, code)
+    L = n_groups * G
+    logits = torch.empty((B, L), dtype=Xt.dtype, device="cuda")
+    H.haste_forward(plan, Xt, Wt, logits, ws)
+    dW = torch.empty((L, k), dtype=Xt.dtype, device="cuda")
+    H.haste_backward_dw(plan, Xt, dYt, dW, ws)
+    dX = torch.full((B, d), float("nan"), dtype=torch.float32, device="cuda")
+    H.haste_backward_dx(plan, Wt, dYt, dX, ws)
+    torch.cuda.synchronize()
+    assert H.haste_device_status() == H.HASTE_OK
+    assert_close(to_np64(logits), O.forward(X, W, idx, G), "logits")
+    assert_close(to_np64(dW), O.backward_dw(X, dY, idx, G), "dW")
+    ref_dx = O.backward_dx(W, dY, idx, G, d)
+    got_dx = to_np64(dX)
+    assert_close(got_dx, ref_dx, "dX")
+    uncovered = np.setdiff1d(np.arange(d), np.unique(idx))
+    assert np.all(got_dx[:, uncovered] == 0.0)
+    # accumulate = 1 adds into the existing dX
+    H.haste_backward_dx(plan, Wt, dYt, dX, ws, accumulate=True)
+    torch.cuda.synchronize()
+    assert_close(to_np64(dX), 2 * ref_dx, "dX accumulated")
+
+
+def test_plan_export_bit_exact_and_index_memory():
+    for (n_groups, k, d, G) in [(256, 32, 256, 16), (20_944, 128, 768, 32)]:
+        idx = I.make_idx(n_groups, k, d, 3)
+        plan = H.haste_plan(idx, G, d)
+        e_idx, off, ent = plan.export()
+        st, r_off, r_ent = O.plan(idx, d)
+        assert np.array_equal(e_idx, idx)
+        assert np.array_equal(off, r_off) and np.array_equal(ent, r_ent)
+        ib, invb = plan.info()
+        assert ib == O.index_bytes(n_groups, k) == 4 * n_groups * k
+        assert ib * G == 4 * n_groups * G * k           # per-label storage would be G times larger
+        assert invb == 4 * (d + 1 + n_groups * k)
+
+
+STEP_CASES = [
+    dict(B=130, d=384, n_groups=250, G=32, k=64, dtype="bf16", H=64, p=5),
+    dict(B=256, d=768, n_groups=300, G=64, k=128, dtype="bf16", H=128, p=8),
+    dict(B=32, d=256, n_groups=256, G=16, k=32, dtype="f32", H=32, p=5),
+    dict(B=300, d=512, n_groups=200, G=16, k=64, dtype="bf16", H=0, p=6),
+]
+
+
+def _step_inputs(c, seed=0):
+    B, d, n_groups, G, k, dt = (c[x] for x in ("B", "d", "n_groups", "G", "k", "dtype"))
+    idx, X, W, _ = _inputs(B, d, n_groups, G, k, dt, seed)
+    L = n_groups * G
+    rp, ids = I.make_zipf_positives(B, c["H"] + L, c["p"], 1.0, seed)
+    (hp, hi), (tp, ti) = I.split_head_tail(rp, ids, c["H"])
+    return idx, X, W, (tp, ti), (hp, hi)
+
+
+def _run_step(plan, X, W, pos, scale):
+    B = X.shape[0]
+    Xt, Wt = to_torch(X), to_torch(W)
+    rp, ids = to_torch(pos[0]), to_torch(pos[1] if len(pos[1]) else np.zeros(1, np.int32))
+    ws = _ws(plan, B, H.dtype_code(Xt))
+    loss = torch.zeros(1, dtype=torch.float32, device="cuda")
+    dW = torch.empty((plan.L, plan.k), dtype=Xt.dtype, device="cuda")
+    dX = torch.full((B, plan.d), float("nan"), dtype=torch.float32, device="cuda")
+    H.haste_bce_step(plan, Xt, Wt, rp, ids, scale, loss, dW, dX, ws)
+    torch.cuda.synchronize()
+    return loss, dW, dX
+
+
+@pytest.mark.parametrize("case", STEP_CASES, ids=lambda c: _case_id(c) + f"_H{c['H']}")
+def test_fused_bce_step(case):
+    idx, X, W, tpos, _ = _step_inputs(case)
+    B, d, G = case["B"], case["d"], case["G"]
+    plan = H.haste_plan(idx, G, d)
+    scale = 1.0 / B
+    loss, dW, dX = _run_step(plan, X, W, tpos, scale)
+    assert H.haste_device_status() == H.HASTE_OK
+    r_loss, _, r_dW, r_dX = O.bce_step(X, W, idx, G, tpos[0], tpos[1], scale)
+    got_loss = float(loss.item())
+    assert abs(got_loss - r_loss) <= 5e-3 * abs(r_loss), (got_loss, r_loss)
+    assert_close(to_np64(dW), r_dW, "dW")
+    assert_close(to_np64(dX), r_dX, "dX")
+    # determinism: a second run gives the same bits
+    loss2, dW2, dX2 = _run_step(plan, X, W, tpos, scale)
+    assert torch.equal(loss, loss2) and torch.equal(dW, dW2) and torch.equal(dX, dX2)
+
+
+HEAD_CASES = [
+    dict(B=256, Hh=384, d=192, dtype="bf16"),
+    dict(B=128, Hh=256, d=128, dtype="f32"),
+    dict(B=256, Hh=4096, d=768, dtype="bf16"),
+]
+
+
+@pytest.mark.parametrize("case", HEAD_CASES, ids=lambda c: "B{B}_H{Hh}_d{d}_{dtype}".format(**c))
+def test_head_forward_backward(case):
+    B, Hh, d, dt = case["B"], case["Hh"], case["d"], case["dtype"]
+    Xh = I.make_normal((B, d), 1.0, 5, 5, dt)
+    Wh = I.make_normal((Hh, d), 1.0 / math.sqrt(d), 5, 6, dt)
+    rp, ids = I.make_zipf_positives(B, Hh, 4, 1.0, 5)
+    Xht, Wht = to_torch(Xh), to_torch(Wh)
+    ws = torch.empty(H.haste_head_workspace_size(B, Hh, d, H.dtype_code(Xht)), dtype=torch.uint8, device="cuda")
+    logits = torch.empty((B, Hh), dtype=Xht.dtype, device="cuda")
+    H.haste_head_forward(Xht, Wht, logits, ws)
+    torch.cuda.synchronize()
+    z = O.head_forward(Xh, Wh)
+    assert_close(to_np64(logits), z, "head logits")
+    # plain-torch fp32 cross-check of the same product
+    ref32 = Xht.float() @ Wht.float().T
+    assert_close(to_np64(logits), ref32.double().cpu().numpy(), "head logits vs torch")
+    dYh = torch.empty_like(logits)
+    loss = torch.zeros(1, dtype=torch.float32, device="cuda")
+    H.haste_head_forward(Xht, Wht, dYh, ws, to_torch(rp), to_torch(ids), 1.0 / B, loss)
+    dWh = torch.empty_like(Wht)
+    dXh = torch.empty((B, d), dtype=torch.float32, device="cuda")
+    H.haste_head_backward(Xht, Wht, dYh, dWh, dXh, ws)
+    torch.cuda.synchronize()
+    r_loss, r_dY, r_dWh, r_dXh = O.head_step(Xh, Wh, rp, ids, 1.0 / B)
+    assert abs(loss.item() - r_loss) <= 5e-3 * abs(r_loss)
+    assert_close(to_np64(dYh), r_dY, "head dY")
+    assert_close(to_np64(dWh), r_dWh, "head dW")
+    assert_close(to_np64(dXh), r_dXh, "head dX")
+
+
+def test_k_equals_d_reduces_to_dense_layer():
+    """idx = [0..d) in every group: the sparse forward is a dense X . W^T."""
+    B, d, n_groups, G = 128, 64, 32, 16
+    idx = np.tile(np.arange(d, dtype=np.int32), (n_groups, 1))
+    X = I.make_normal((B, d), 1.0, 9, 1, "bf16")
+    W = I.make_normal((n_groups * G, d), 0.125, 9, 2, "bf16")
+    plan = H.haste_plan(idx, G, d)
+    Xt, Wt = to_torch(X), to_torch(W)
+    ws = _ws(plan, B, H.HASTE_BF16)
+    out = torch.empty((B, n_groups * G), dtype=torch.bfloat16, device="cuda")
+    H.haste_forward(plan, Xt, Wt, out, ws)
+    torch.cuda.synchronize()
+    ref = (Xt.float() @ Wt.float().T).double().cpu().numpy()
+    assert_close(to_np64(out), ref, "dense special case")
+
+
+def test_error_statuses():
+    idx = I.make_idx(64, 64, 256, 1)
+    plan = H.haste_plan(idx, 16, 256)
+    X = torch.zeros((32, 256), dtype=torch.bfloat16, device="cuda")
+    W = torch.zeros((64 * 16, 64), dtype=torch.bfloat16, device="cuda")
+    out = torch.empty((32, 64 * 16), dtype=torch.bfloat16, device="cuda")
+    small = torch.empty(16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(H.HasteError) as e:
+        H.haste_forward(plan, X, W, out, small)
+    assert e.value.status == H.HASTE_ERR_WORKSPACE
+    bad = H.haste_plan(I.make_idx(8, 48, 256, 1), 16, 256)       # k*2 bytes not a multiple of 128
+    Wb = torch.zeros((8 * 16, 48), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(H.HasteError) as e:
+        H.haste_forward(bad, X, Wb, torch.empty((32, 128), dtype=torch.bfloat16, device="cuda"), None)
+    assert e.value.status == H.HASTE_ERR_UNSUPPORTED_SHAPE
+    with pytest.raises(H.HasteError) as e:
+        H.haste_plan(np.array([[0, 0]], dtype=np.int32), 16, 8)
+    assert e.value.status == H.HASTE_ERR_INDEX_UNSORTED_OR_DUP
+
+
+def test_bounded_wait_timeout_is_reported_and_context_survives():
+    assert H.haste_device_status() == H.HASTE_OK
+    assert H.lib().haste_selftest_wait_timeout(H._stream(None)) == H.HASTE_OK
+    assert H.haste_device_status() == H.HASTE_ERR_TIMEOUT
+    assert H.haste_device_status() == H.HASTE_OK          # cleared after reporting
+    a = torch.ones(1024, device="cuda")
+    assert float((a * 2).sum().item()) == 2048.0
