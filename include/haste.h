@@ -158,6 +158,29 @@ haste_status_t haste_backward_dx(haste_plan_t plan, int32_t B, haste_dtype_t dty
                                  const void* dY, float* dX, int accumulate, void* ws, size_t ws_bytes,
                                  haste_stream_t stream);
 
+/* dX like haste_backward_dx, for callers that must not allocate device memory:
+ * no workspace argument, and the call makes no cudaMalloc, cudaFree or other
+ * allocating call.  Such callers include code running under a framework whose
+ * caching allocator has reserved the device memory (a raw cudaMalloc can fail or
+ * fragment that pool), hooks that run inside another library's call path, and
+ * loops that are not allowed to allocate at all.  The paper has no counterpart;
+ * this is a deployment variant of the dX reduction.
+ *   Scratch: a file-scope static device array of 16 MiB (16777216 bytes) holds
+ *   the reduction's per-chunk partials; every GPU that loads the library keeps it
+ *   until the process exits.  The partials are fully rewritten by each call, so
+ *   nothing in it needs clearing.  All calls share this one array: calls whose
+ *   kernels overlap on the GPU (other streams, other host threads) race on it and
+ *   give wrong results; serialise them.
+ *   Limit: d * roundup(B, 128) * 4 must not exceed 16 MiB (one chunk of
+ *   partials); larger shapes return HASTE_ERR_UNSUPPORTED_SHAPE with a message.
+ *   Fewer group chunks may be used than in haste_backward_dx, so the two can
+ *   differ in the rounding of the chunk sums (both are deterministic).
+ *   Set-up: the first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call before
+ *   any stream capture. */
+haste_status_t haste_backward_dx_noalloc(haste_plan_t plan, int32_t B, haste_dtype_t dtype, const void* W,
+                                         const void* dY, float* dX, int accumulate, haste_stream_t stream);
+
 /* Fused tail training step (logits never reach global memory):
  *   z = forward(X, W);  y[b,l] = 1 iff l is in tail_pos row b;
  *   dY = grad_scale * (sigmoid(z) - y)   (rounded to the input dtype);

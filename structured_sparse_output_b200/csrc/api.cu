@@ -209,6 +209,32 @@ cudaError_t xt(const TailArgs& a, const void* X, void* Xt, cudaStream_t st) {
   return tail::launch_xt<T>(X, Xt, a.sh.B, a.sh.Bp, a.sh.d, st);
 }
 
+// Scratch of haste_backward_dx_noalloc: static device memory (no allocation at
+// call time).  Holds the per-chunk dX partials; every GPU that loads the library
+// keeps these bytes until the process exits.
+constexpr size_t kNoAllocScratchBytes = (size_t)16 << 20;
+__device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of g_noalloc_scratch, looked up once per device (host code only
+// sees a host-side stand-in under that name).
+constexpr int kMaxDevices = 64;
+void* g_noalloc_addr[kMaxDevices] = {};
+std::mutex g_noalloc_mu;
+
+haste_status_t noalloc_scratch(void** out) {
+  int dev = 0;
+  HASTE_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDevices) return fail(HASTE_ERR_INVALID_ARG, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> g(g_noalloc_mu);
+  if (!g_noalloc_addr[dev]) {
+    void* p = nullptr;
+    HASTE_CUDA(cudaGetSymbolAddress(&p, g_noalloc_scratch));
+    g_noalloc_addr[dev] = p;
+  }
+  *out = g_noalloc_addr[dev];
+  return HASTE_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -501,6 +527,44 @@ haste_status_t haste_backward_dx(haste_plan_t p, int32_t B, haste_dtype_t dt, co
     e = tail::launch_dx_reduce(a.dX_part, dX, t.n_chunks, p->d, a.sh.Bp, B, accumulate, s);
   }
   return e == cudaSuccess ? HASTE_OK : cuda_fail(e, "haste_backward_dx launch");
+}
+
+// dX without a workspace and without any allocation: the chunk partials live in
+// the library's static scratch (16 MiB), so the group chunks of the reduction
+// are capped to what fits there.  Same result definition as haste_backward_dx;
+// the cap can change the chunking and hence the rounding of the chunk sums.
+haste_status_t haste_backward_dx_noalloc(haste_plan_t p, int32_t B, haste_dtype_t dt, const void* W, const void* dY,
+                                         float* dX, int accumulate, haste_stream_t stream) {
+  DeviceInfo di;
+  haste_status_t st = device_info(di);
+  if (st == HASTE_OK) st = check_tail(p, B, dt, di);
+  if (st != HASTE_OK) return st;
+  if (!W || !dY || !dX) return fail(HASTE_ERR_INVALID_ARG, "NULL tensor pointer");
+  const int E = elem_bytes(dt);
+  const int Bp = round_up(B, 128);
+  DxTiling t = dx_tiling(*p, Bp, E, di.sms, di.smem_optin);
+  const size_t per_chunk = (size_t)p->d * Bp * 4;
+  const size_t max_chunks = kNoAllocScratchBytes / per_chunk;
+  if (max_chunks < 1)
+    return fail(HASTE_ERR_UNSUPPORTED_SHAPE,
+                "haste_backward_dx_noalloc needs d*roundup(B,128)*4 = %zu bytes of scratch; its static scratch "
+                "holds %zu bytes",
+                per_chunk, kNoAllocScratchBytes);
+  if ((size_t)t.n_chunks > max_chunks) t.n_chunks = (int)max_chunks;
+  void* scratch = nullptr;
+  if ((st = noalloc_scratch(&scratch)) != HASTE_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  TailArgs a = make_args(*p, B);
+  a.W = W;
+  a.dY = dY;
+  a.dX_part = static_cast<float*>(scratch);
+  a.band = t.band;
+  a.n_bands = t.n_bands;
+  a.n_chunks = t.n_chunks;
+  cudaError_t e = dt == HASTE_BF16 ? tail::launch_backward_dx<__nv_bfloat16>(a, false, s)
+                                   : tail::launch_backward_dx<float>(a, false, s);
+  if (e == cudaSuccess) e = tail::launch_dx_reduce(a.dX_part, dX, t.n_chunks, p->d, Bp, B, accumulate, s);
+  return e == cudaSuccess ? HASTE_OK : cuda_fail(e, "haste_backward_dx_noalloc launch");
 }
 
 haste_status_t haste_bce_step(haste_plan_t p, int32_t B, haste_dtype_t dt, const void* X, const void* W,

@@ -75,6 +75,7 @@ def lib() -> ctypes.CDLL:
         "haste_forward": ([P, I32, S, P, P, P, P, SZ, P], S),
         "haste_backward_dw": ([P, I32, S, P, P, P, P, SZ, P], S),
         "haste_backward_dx": ([P, I32, S, P, P, P, S, P, SZ, P], S),
+        "haste_backward_dx_noalloc": ([P, I32, S, P, P, P, S, P], S),
         "haste_bce_step": ([P, I32, S, P, P, Targets, F, P, P, P, S, P, SZ, P], S),
         "haste_head_workspace_size": ([I32, I32, I32, S], SZ),
         "haste_head_forward": ([I32, I32, I32, S, P, P, P, P, F, P, P, SZ, P], S),
@@ -216,6 +217,12 @@ def haste_backward_dx(plan: Plan, W, dY, dX, ws, accumulate: bool = False, strea
     p, n = _ws(ws)
     _check(lib().haste_backward_dx(plan.handle, dY.shape[0], dtype_code(W), _tptr(W), _tptr(dY), _tptr(dX),
                                    int(accumulate), p, n, _stream(stream)), "haste_backward_dx")
+
+
+def haste_backward_dx_noalloc(plan: Plan, W, dY, dX, accumulate: bool = False, stream=None) -> None:
+    """dX with no workspace and no device allocation (library-owned static scratch)."""
+    _check(lib().haste_backward_dx_noalloc(plan.handle, dY.shape[0], dtype_code(W), _tptr(W), _tptr(dY), _tptr(dX),
+                                           int(accumulate), _stream(stream)), "haste_backward_dx_noalloc")
 
 
 def haste_bce_step(plan: Plan, X, W, pos_row_ptr, pos_ids, grad_scale: float, loss, dW, dX, ws,
