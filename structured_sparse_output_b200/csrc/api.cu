@@ -18,6 +18,7 @@
 
 #include "head.cu"
 #include "tail.cu"
+#include "tail_v2.cu"
 
 using namespace haste;
 
@@ -126,15 +127,21 @@ struct DxTiling {
   int band, n_bands, n_chunks;
 };
 
+// The warp-specialised TMA kernels cover bf16 with G in {16, 32, 64}, k in
+// {64, 128} and at most two 128-row batch tiles; other shapes run the staged
+// kernels of tail.cu.
+bool use_v2(const haste_plan_s& p, int Bp, int elem) { return elem == 2 && tail2::supported(p.G, p.k, Bp); }
+
 DxTiling dx_tiling(const haste_plan_s& p, int Bp, int elem, int sms, int smem_optin) {
   DxTiling t{};
-  const size_t fixed = tail::smem_dx(elem, p.k, p.G, 0);
-  long avail = (long)smem_optin - (long)fixed;
-  int band = (int)std::min<long>(256, avail / 512);
+  const size_t fixed = use_v2(p, Bp, elem) ? tail2::dx_smem(0, p.k, p.G) : tail::smem_dx(elem, p.k, p.G, 0);
+  long avail = (long)smem_optin - (long)fixed - 4096;  // headroom for static shared memory
+  int band = (int)std::min<long>(use_v2(p, Bp, elem) ? 512 : 256, avail / 512);
   band = std::max(8, band & ~7);
   if (band > p.d) band = round_up(p.d, 8);
-  t.band = band;
+  // as few bands as fit, then split d evenly between them
   t.n_bands = (p.d + band - 1) / band;
+  t.band = round_up((p.d + t.n_bands - 1) / t.n_bands, 8);
   const int per_chunk = (Bp / 128) * t.n_bands;
   int c = std::max(1, sms / per_chunk);
   if ((int64_t)c > p.n_groups) c = (int)p.n_groups;
@@ -157,8 +164,8 @@ TailWs tail_ws(const haste_plan_s& p, int B, int elem, const DxTiling& t) {
   off = align256(off + (size_t)p.d * Bp * elem);
   w.dx_part = off;
   off = align256(off + (size_t)t.n_chunks * p.d * Bp * 4);
-  w.dy_buf = off;
-  off = align256(off + (size_t)B * p.n_groups * p.G * elem);
+  w.dy_buf = off;  // [B, L] (staged kernels) or group-major [n_groups, Bp, G]
+  off = align256(off + (size_t)Bp * p.n_groups * p.G * elem);
   w.loss_part = off;
   off = align256(off + (size_t)kMaxLossParts * 4);
   w.total = off;
@@ -202,6 +209,23 @@ TailArgs make_args(const haste_plan_s& p, int B) {
   a.sh.L = p.n_groups * p.G;
   a.idx = p.idx_d;
   return a;
+}
+
+// dX pass through the pipelined bf16 kernel.  Element (b, g*G + j) of dY sits at
+// dY[g*gstride + b*rstride + j]: (G, L) for the caller's [B, L] gradient,
+// (Bp*G, G) for the fused step's group-major buffer.
+cudaError_t dx_v2(const haste_plan_s& p, int B, const void* W, const void* dY, int64_t gstride, int64_t rstride,
+                  float* part, const DxTiling& t, cudaStream_t s) {
+  v2::DxArgs a{};
+  a.sh = make_args(p, B).sh;
+  a.idx = p.idx_d;
+  a.dX_part = part;
+  a.band = t.band;
+  a.n_bands = t.n_bands;
+  a.n_chunks = t.n_chunks;
+  a.dy_gstride = gstride;
+  a.dy_rstride = rstride;
+  return tail2::launch_dx(p.G, p.k, a, dY, W, s);
 }
 
 template <typename T>
@@ -519,8 +543,11 @@ haste_status_t haste_backward_dx(haste_plan_t p, int32_t B, haste_dtype_t dt, co
   cudaError_t e;
   {
     ProfScope ps("tail_dx", s);
-    e = dt == HASTE_BF16 ? tail::launch_backward_dx<__nv_bfloat16>(a, false, s)
-                         : tail::launch_backward_dx<float>(a, false, s);
+    if (use_v2(*p, a.sh.Bp, E))
+      e = dx_v2(*p, B, W, dY, p->G, a.sh.L, a.dX_part, t, s);
+    else
+      e = dt == HASTE_BF16 ? tail::launch_backward_dx<__nv_bfloat16>(a, false, s)
+                           : tail::launch_backward_dx<float>(a, false, s);
   }
   if (e == cudaSuccess) {
     ProfScope ps("dx_reduce", s);
@@ -561,8 +588,9 @@ haste_status_t haste_backward_dx_noalloc(haste_plan_t p, int32_t B, haste_dtype_
   a.band = t.band;
   a.n_bands = t.n_bands;
   a.n_chunks = t.n_chunks;
-  cudaError_t e = dt == HASTE_BF16 ? tail::launch_backward_dx<__nv_bfloat16>(a, false, s)
-                                   : tail::launch_backward_dx<float>(a, false, s);
+  cudaError_t e = use_v2(*p, Bp, E) ? dx_v2(*p, B, W, dY, p->G, a.sh.L, a.dX_part, t, s)
+                 : dt == HASTE_BF16  ? tail::launch_backward_dx<__nv_bfloat16>(a, false, s)
+                                     : tail::launch_backward_dx<float>(a, false, s);
   if (e == cudaSuccess) e = tail::launch_dx_reduce(a.dX_part, dX, t.n_chunks, p->d, Bp, B, accumulate, s);
   return e == cudaSuccess ? HASTE_OK : cuda_fail(e, "haste_backward_dx_noalloc launch");
 }
@@ -599,7 +627,9 @@ haste_status_t haste_bce_step(haste_plan_t p, int32_t B, haste_dtype_t dt, const
   a.band = t.band;
   a.n_bands = t.n_bands;
   a.n_chunks = t.n_chunks;
-  const int grid = dt == HASTE_BF16 ? tail::step_grid<__nv_bfloat16>(a, di.sms) : tail::step_grid<float>(a, di.sms);
+  const bool v2p = use_v2(*p, Bp, E) && tail2::step_smem(Bp, p->k, p->G) <= (size_t)di.smem_optin;
+  const int grid = v2p ? (int)std::min<int64_t>(p->n_groups, di.sms)
+                       : dt == HASTE_BF16 ? tail::step_grid<__nv_bfloat16>(a, di.sms) : tail::step_grid<float>(a, di.sms);
   if (grid <= 0 || grid > kMaxLossParts) return fail(HASTE_ERR_CUDA, "could not size the fused step grid");
   cudaError_t e;
   {
@@ -609,12 +639,30 @@ haste_status_t haste_bce_step(haste_plan_t p, int32_t B, haste_dtype_t dt, const
   }
   if (e == cudaSuccess) {
     ProfScope ps("tail_step", s);
-    e = dt == HASTE_BF16 ? tail::launch_step<__nv_bfloat16>(a, grid, s) : tail::launch_step<float>(a, grid, s);
+    if (v2p) {
+      v2::StepArgs sa{};
+      sa.sh = a.sh;
+      sa.idx = p->idx_d;
+      sa.dW = static_cast<__nv_bfloat16*>(dW);
+      sa.dY_out = static_cast<__nv_bfloat16*>(a.dY_out);
+      sa.loss_part = a.loss_part;
+      sa.pos_ptr = pos.row_ptr;
+      sa.pos_ids = pos.ids;
+      sa.grad_scale = grad_scale;
+      e = tail2::launch_step(p->G, p->k, sa, grid, a.Xt, W, s);
+    } else {
+      e = dt == HASTE_BF16 ? tail::launch_step<__nv_bfloat16>(a, grid, s) : tail::launch_step<float>(a, grid, s);
+    }
   }
   if (e == cudaSuccess) {
     ProfScope ps("tail_dx", s);
-    e = dt == HASTE_BF16 ? tail::launch_backward_dx<__nv_bfloat16>(a, true, s)
-                         : tail::launch_backward_dx<float>(a, true, s);
+    if (v2p)
+      e = dx_v2(*p, B, W, a.dY_out, (int64_t)Bp * p->G, p->G, a.dX_part, t, s);
+    else if (use_v2(*p, Bp, E))
+      e = dx_v2(*p, B, W, a.dY_out, p->G, a.sh.L, a.dX_part, t, s);
+    else
+      e = dt == HASTE_BF16 ? tail::launch_backward_dx<__nv_bfloat16>(a, true, s)
+                           : tail::launch_backward_dx<float>(a, true, s);
   }
   if (e == cudaSuccess) {
     ProfScope ps("dx_reduce", s);

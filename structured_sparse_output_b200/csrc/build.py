@@ -14,7 +14,7 @@ SOURCES = ["api.cu", "tail.cu", "head.cu", "common.cuh", "tail.cuh",
            os.path.join("..", "..", "include", "haste.h")]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",
-         "--expt-relaxed-constexpr", "-Xcompiler", "-fPIC,-O2", "-shared"]
+         "--expt-relaxed-constexpr", "-maxrregcount=152", "-Xcompiler", "-fPIC,-O2", "-shared"]
 
 
 def stale() -> bool:

@@ -4,6 +4,7 @@
 // tensor cores.  Everything is inline PTX written for this library.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -73,11 +74,40 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64
   return false;
 }
 
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+
+// ------------------------------------------------------------------- TMA
+// 2D tiled load of one box at coordinates (c0 = innermost, c1) into shared
+// memory; completion is signalled on the mbarrier as transaction bytes.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* tm, int c0, int c1, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(
+          dst),
+      "l"(tm), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
+      : "memory");
+}
+// Four rows r0..r3 (arbitrary) of a 2D tensor, columns [col, col + box width),
+// written as four consecutive box rows at dst.
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* tm, int col, int r0, int r1, int r2, int r3,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(dst),
+      "l"(tm), "r"(smem_u32(bar)), "r"(col), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
+      : "memory");
+}
+
 // ---------------------------------------------------------------- cp.async
 // 16-byte global->shared copy through L2 only; src_bytes < 16 zero-fills the rest.
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
                : "memory");
+}
+// Named barrier over a subset of warps (ids 1..15; id 0 is __syncthreads).
+__device__ __forceinline__ void named_bar(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
@@ -97,6 +127,14 @@ __device__ __forceinline__ uint32_t sw128(uint32_t off) { return off ^ (((off >>
 // 4 rows of 128 B per 512-byte atom): the shared-memory layout that MN-major
 // tf32 operands of tcgen05.mma require.
 __device__ __forceinline__ uint32_t sw128_32b(uint32_t off) { return off ^ (((off >> 7) & 3u) << 5); }
+
+// Swizzle of rows of rb = 32, 64 or 128 bytes inside a 1024-byte aligned region
+// (16-byte chunk index XOR bits 7.. of the offset), the pattern of the TMA and
+// UMMA 32B / 64B / 128B swizzle modes.
+__device__ __forceinline__ uint32_t swz_rows(uint32_t off, int rb) {
+  const uint32_t m = (uint32_t)(rb / 16 - 1);
+  return off ^ (((off >> 7) & m) << 4);
+}
 
 // Swizzle of a 128B-row tile for element type T read as a K-major (kMN = false)
 // or MN-major (kMN = true) operand.
@@ -162,11 +200,25 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
 #pragma unroll
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
+// 32 lanes x 8 consecutive 32-bit columns.
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float* v) {
+  uint32_t r[8];
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+}
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 // ------------------------------------------------------------- descriptors
 // Layout codes of the shared-memory matrix descriptor (bits 61..63).
-enum : uint32_t { kLayoutNone = 0, kLayoutSw128Base32 = 1, kLayoutSw128 = 2 };
+enum : uint32_t { kLayoutNone = 0, kLayoutSw128Base32 = 1, kLayoutSw128 = 2, kLayoutSw64 = 4, kLayoutSw32 = 6 };
+
+// Descriptor layout code of rows of rb bytes (128, 64 or 32).
+__host__ __device__ constexpr uint32_t layout_for_rows(int rb) {
+  return rb == 128 ? kLayoutSw128 : rb == 64 ? kLayoutSw64 : kLayoutSw32;
+}
 
 // Shared-memory matrix descriptor: start address, leading-dimension byte offset
 // (LBO), stride-dimension byte offset (SBO), descriptor version 1 (bit 46) and

@@ -1,0 +1,678 @@
+// tail_v2.cu -- warp-specialised, pipelined bf16 kernels of the group-shared sparse
+// tail (HASTE, "Hardware-Aware Dynamic Sparse Training for Large Output Spaces",
+// Methodology 1: labels in groups of G share one fan-in set I_g of k features).
+//
+// k_step2 -- fused forward + BCE gradient + dW, one group per iteration:
+//   warps 0-1  producers: the gather-once tile X[:, I_g] (k rows of X^T) and the
+//              G x k weight block, staged with cp.async into a 2-stage ring; warp
+//              0 owns stage 0 and warp 1 stage 1;
+//   warp 2     MMA issuer (one thread): forward of group i+1 is issued before the
+//              dW of group i, so the tensor core works while the epilogue runs;
+//   warps 3-10 epilogue: logits leave TMEM only as the BCE gradient (bf16, to
+//              shared memory for the dW product and to the group-major gradient
+//              buffer of the dX pass), then dW is read out of TMEM.
+// k_dx2 -- dX pass: per CTA (128-row batch tile, feature band, group chunk):
+//   warps 0-3 stage the dY tile and the weight columns of the band's slots
+//   (multi-stage ring; warp 0 also writes the slot metadata into an 8-entry ring),
+//   warp 4 issues Z = dY_g . W_g[:, slots], warps 5-20 add the rows of Z into a
+//   fp32 band accumulator in shared memory.  Scatter warp (q, p) owns batch rows
+//   [32q, 32q+32) and the p-th quarter of the band's features, so every feature
+//   receives its group terms in ascending group order, deterministically.
+#include "tail.cuh"
+
+namespace haste {
+namespace v2 {
+
+struct StepArgs {
+  TailShape sh;
+  const int32_t* idx;
+  __nv_bfloat16* dW;
+  __nv_bfloat16* dY_out;  // group-major gradient buffer [n_groups, Bp, G]
+  float* loss_part;
+  const int32_t* pos_ptr;
+  const int32_t* pos_ids;
+  float grad_scale;
+};
+
+struct DxArgs {
+  TailShape sh;
+  const int32_t* idx;
+  float* dX_part;
+  int band, n_bands, n_chunks;
+  // element (b, g*G + j) of dY is at dY[g*dy_gstride + b*dy_rstride + j]
+  int64_t dy_gstride, dy_rstride;
+};
+
+constexpr int kMetaSlots = 8;  // metadata ring of the dX pass
+constexpr int kMetaHdr = 8;    // 5 slot split points, s0, N, 1 spare
+
+template <int kG>
+__host__ __device__ constexpr int dx_stages() {
+  return kG <= 32 ? 4 : 3;
+}
+
+// ------------------------------------------------------------ smem layouts
+struct StepLayout {
+  uint32_t xg[2], wg[2], dy[2], bars, total;
+};
+__host__ __device__ inline StepLayout step_layout(int Bp, int k, int G) {
+  StepLayout L;
+  const uint32_t xg = (uint32_t)((Bp / 64) * k * 128 + (k < 128 ? (128 - k) * 128 : 0));
+  const uint32_t wg = (uint32_t)((k / 64) * G * 128);
+  const uint32_t dy = (uint32_t)(Bp * G * 2);
+  uint32_t off = 0;
+  for (int s = 0; s < 2; ++s) { L.xg[s] = off; off += xg; }
+  for (int s = 0; s < 2; ++s) { L.wg[s] = off; off += wg; }
+  for (int s = 0; s < 2; ++s) { L.dy[s] = off; off += (dy + 1023u) & ~1023u; }
+  L.bars = off;
+  off += 256;
+  L.total = off + 1024;
+  return L;
+}
+
+struct DxLayout {
+  uint32_t dy, w, acc, meta, bars, total, dy_stride, w_stride, meta_stride;
+};
+__host__ __device__ inline DxLayout dx_layout(int band, int k, int G, int ns) {
+  DxLayout L;
+  L.dy_stride = (uint32_t)((128 * G * 2 + 1023) & ~1023);
+  L.w_stride = (uint32_t)((k / 64) * G * 128);
+  L.meta_stride = (uint32_t)(kMetaHdr + k) * 4;
+  uint32_t off = 0;
+  L.dy = off;
+  off += ns * L.dy_stride;
+  L.w = off;
+  off += ns * L.w_stride;
+  L.acc = off;
+  off += (uint32_t)band * 128 * 4;
+  L.meta = off;
+  off += kMetaSlots * L.meta_stride;
+  off = (off + 7) & ~7u;
+  L.bars = off;
+  off += 512;
+  L.total = off + 1024;
+  return L;
+}
+
+__device__ __forceinline__ int warp_id() { return threadIdx.x >> 5; }
+__device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
+
+// Bounded wait; on timeout the CTA-wide abort flag is raised.
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  if (*abort_flag) return false;
+  if (!mbar_wait(bar, parity)) {
+    *abort_flag = 1;
+    return false;
+  }
+  return true;
+}
+
+// A producer thread publishes its finished copies to the tensor core (proxy
+// fence) before arriving on the stage's full barrier.
+__device__ __forceinline__ void publish_all(uint64_t* full_bar) {
+  cp_async_wait_all();
+  fence_proxy_async_smem();
+  mbar_arrive(full_bar);
+}
+
+// ============================================================ k_step2
+constexpr int kStepThreads = 352;  // 2 producer warps, MMA warp, 8 epilogue warps (<= 3 per scheduler)
+constexpr int kMaxPosReg = 8;      // positives per batch row kept in registers
+
+template <int kG, int kK>
+__global__ void __launch_bounds__(kStepThreads, 1)
+    k_step2(StepArgs a, const __nv_bfloat16* __restrict__ Xt, const __nv_bfloat16* __restrict__ W) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  constexpr int RB = kG * 2;   // bytes of one dY row in shared memory
+  constexpr int CH = kG / 2;   // label columns per epilogue half
+  constexpr int kRowsPerThr = kK / 4;
+  const TailShape sh = a.sh;
+  const int Bp = sh.Bp, n_bt = Bp / 128;
+  const StepLayout Lo = step_layout(Bp, kK, kG);
+  const uint32_t base = align1024(smem_u32(smem));
+  uint8_t* gbase = smem + (base - smem_u32(smem));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(gbase + Lo.bars);
+  uint64_t* full = bars;             // [2] stage loaded (count: one producer half)
+  uint64_t* empty = bars + 2;        // [2] stage free
+  uint64_t* fwd_full = bars + 4;     // [2] logits in TMEM
+  uint64_t* dy_full = bars + 6;      // [2] dY in shared memory
+  uint64_t* dw_full = bars + 8;      // [2] dW in TMEM
+  uint64_t* tmem_empty = bars + 10;  // [2] TMEM buffer read out
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 12);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
+  float* red = reinterpret_cast<float*>(tslot + 2);  // 8 warp partials
+
+  const int w = warp_id(), lane = lane_id();
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&full[s], 32);
+      mbar_init(&empty[s], 1);
+      mbar_init(&fwd_full[s], 1);
+      mbar_init(&dy_full[s], 8);
+      mbar_init(&dw_full[s], 1);
+      mbar_init(&tmem_empty[s], 8);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  // TMEM: forward accumulators F[2] (n_bt*G columns each), dW accumulators D[2]
+  const uint32_t f_cols = (uint32_t)(n_bt * kG);
+  const uint32_t ncols = tmem_cols_for(2 * f_cols + 2 * kG);
+  if (w == 2) {
+    tmem_alloc(tslot, ncols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tslot;
+  auto F = [&](int s) -> uint32_t { return tmem + (s ? f_cols : 0u); };
+  auto D = [&](int s) -> uint32_t { return tmem + 2 * f_cols + (s ? (uint32_t)kG : 0u); };
+  auto XG = [&](int s) -> uint32_t { return base + (s ? Lo.xg[1] : Lo.xg[0]); };
+  auto WG = [&](int s) -> uint32_t { return base + (s ? Lo.wg[1] : Lo.wg[0]); };
+  auto DY = [&](int s) -> uint32_t { return s ? Lo.dy[1] : Lo.dy[0]; };
+
+  // contiguous chunk of groups per CTA
+  const int64_t gb = (int64_t)blockIdx.x * sh.n_groups / gridDim.x;
+  const int64_t ge = (int64_t)(blockIdx.x + 1) * sh.n_groups / gridDim.x;
+  const int n_items = (int)(ge - gb);
+
+  if (w < 2) {
+    // ------------------------------------------------- cp.async producers
+    // warp h fills stage h with the items i = h, h+2, ...  Lane (rg, sub) copies
+    // the 16-byte chunk sub of every 128-byte segment of the rows rg, rg+4, ...
+    // so that 8 consecutive lanes read one segment; the feature indices of its
+    // rows sit in registers.
+    const int half = w, ht = lane;
+    const int sub = ht & 7, rg = ht >> 3;
+    const uint32_t xg = XG(half), wg = WG(half);
+    int i = half;
+    for (; i < n_items; i += 2) {
+      const int64_t g = gb + i;
+      // the index loads are in flight while this half waits for its stage
+      int idx_cur[kRowsPerThr];
+#pragma unroll
+      for (int m = 0; m < kRowsPerThr; ++m) idx_cur[m] = a.idx[g * kK + rg + 4 * m];
+      if (!wait_or_abort(&empty[half], ((i >> 1) & 1) ^ 1, abort_flag)) break;
+      const int nbb = Bp / 64;
+#pragma unroll
+      for (int m = 0; m < kRowsPerThr; ++m) {
+        const int sl = rg + 4 * m;
+        const __nv_bfloat16* src = Xt + (int64_t)idx_cur[m] * Bp + sub * 8;
+        const uint32_t dst = xg + sw128((uint32_t)(sl * 128 + sub * 16));  // swizzle is the same in every block
+#pragma unroll
+        for (int bb = 0; bb < 4; ++bb)
+          if (bb < nbb) cp_async16(dst + (uint32_t)(bb * kK * 128), src + bb * 64, 16);
+      }
+      // weight block of the group (contiguous G x k)
+      const __nv_bfloat16* wsrc = W + g * (int64_t)kG * kK;
+      constexpr int cpr = kK / 8;
+#pragma unroll 4
+      for (int c0 = 0; c0 < kG * cpr; c0 += 32) {
+        const int c = c0 + ht;
+        const int j = c / cpr, cc = c % cpr;
+        cp_async16(wg + sw128((uint32_t)((cc >> 3) * kG * 128 + j * 128 + (cc & 7) * 16)),
+                   wsrc + (int64_t)j * kK + cc * 8, 16);
+      }
+      cp_async_commit();
+      publish_all(&full[half]);
+    }
+    cp_async_wait_all();
+  } else if (w == 2) {
+    // ------------------------------------------------------------ MMA issuer
+    const uint32_t idesc_f = make_idesc(1, 1, 0, 128, kG);
+    const uint32_t idesc_w = make_idesc(1, 0, 1, 128, kG);
+    auto issue_fwd = [&](int i) -> bool {
+      const int s = i & 1;
+      if (!wait_or_abort(&tmem_empty[s], ((i >> 1) & 1) ^ 1, abort_flag)) return false;
+      if (!wait_or_abort(&full[s], (i >> 1) & 1, abort_flag)) return false;
+      tc_fence_after();
+      if (lane == 0) {
+        for (int t = 0; t < n_bt; ++t)
+          for (int kk = 0; kk < kK / 16; ++kk) {
+            const uint64_t ad = make_sdesc(XG(s) + (uint32_t)(t * 2 * kK * 128 + kk * 16 * 128), (uint32_t)kK * 128,
+                                           1024, kLayoutSw128);
+            const uint64_t bd =
+                make_sdesc(WG(s) + (uint32_t)((kk / 4) * kG * 128 + (kk % 4) * 32), 16, 1024, kLayoutSw128);
+            mma_ss<false>(F(s) + (uint32_t)(t * kG), ad, bd, idesc_f, kk > 0 ? 1u : 0u);
+          }
+        mma_commit(&fwd_full[s]);
+      }
+      __syncwarp();
+      return true;
+    };
+    bool ok = n_items > 0 ? issue_fwd(0) : true;
+    for (int i = 0; ok && i < n_items; ++i) {
+      if (i + 1 < n_items && !issue_fwd(i + 1)) break;
+      const int s = i & 1;
+      if (!wait_or_abort(&dy_full[s], (i >> 1) & 1, abort_flag)) break;
+      tc_fence_after();
+      if (lane == 0) {
+        for (int kk = 0; kk < Bp / 16; ++kk) {
+          const int b = kk * 16;
+          const uint64_t ad =
+              make_sdesc(XG(s) + (uint32_t)((b / 64) * kK * 128 + (kk % 4) * 32), 16, 1024, kLayoutSw128);
+          const uint64_t bd = make_sdesc(base + DY(s) + (uint32_t)(b * RB), 16, 8 * RB, layout_for_rows(RB));
+          mma_ss<false>(D(s), ad, bd, idesc_w, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&dw_full[s]);
+        mma_commit(&empty[s]);
+      }
+      __syncwarp();
+    }
+  } else {
+    // ------------------------------------------------------------- epilogue
+    // warp (q, hh): TMEM lane quarter q, label columns [hh*CH, hh*CH + CH)
+    const int ew = w - 3, q = w & 3, hh = ew >> 2;
+    const int r = q * 32 + lane;  // row inside a 128-row tile (and dW slot)
+    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    const float scale = a.grad_scale;
+    float loss_acc = 0.f;
+    // this thread's positives (tail-local ids), one batch row per 128-row tile
+    int pos[2][kMaxPosReg];
+    int npos[2] = {0, 0}, pbeg[2] = {0, 0};
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      const int b = t * 128 + r;
+      if (t < n_bt && b < sh.B) {
+        pbeg[t] = a.pos_ptr[b];
+        npos[t] = a.pos_ptr[b + 1] - pbeg[t];
+      }
+#pragma unroll
+      for (int e = 0; e < kMaxPosReg; ++e) pos[t][e] = e < npos[t] ? a.pos_ids[pbeg[t] + e] : -1;
+    }
+    for (int i = 0; i < n_items; ++i) {
+      const int64_t g = gb + i;
+      const int s = i & 1;
+      if (!wait_or_abort(&fwd_full[s], (i >> 1) & 1, abort_flag)) break;
+      tc_fence_after();
+      const int64_t l0 = g * kG + hh * CH;  // first label of this warp's columns
+      uint8_t* dyrow = gbase + DY(s);
+      __nv_bfloat16* dyg = a.dY_out + g * (int64_t)Bp * kG;
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        if (t >= n_bt) break;
+        const int b = t * 128 + r;
+        const bool live = b < sh.B;
+        uint32_t ym = 0;
+#pragma unroll
+        for (int e = 0; e < kMaxPosReg; ++e) {
+          const int64_t l = (int64_t)pos[t][e] - l0;
+          if (pos[t][e] >= 0 && l >= 0 && l < CH) ym |= 1u << l;
+        }
+        for (int e = kMaxPosReg; e < npos[t]; ++e) {  // rows with many positives
+          const int64_t l = (int64_t)a.pos_ids[pbeg[t] + e] - l0;
+          if (l >= 0 && l < CH) ym |= 1u << l;
+        }
+#pragma unroll
+        for (int c = 0; c < CH; c += 16) {
+          constexpr int NC = CH < 16 ? CH : 16;
+          float z[16];
+          if constexpr (NC == 8) tmem_ld8(F(s) + lane_off + (uint32_t)(t * kG + hh * CH + c), z);
+          else tmem_ld16(F(s) + lane_off + (uint32_t)(t * kG + hh * CH + c), z);
+          tmem_wait_ld();
+          float dyv[16], lin = 0.f, prod = 1.f;
+#pragma unroll
+          for (int e = 0; e < NC; ++e) {
+            const float y = ((ym >> (c + e)) & 1u) ? 1.f : 0.f;
+            const float th = tanh_approx(0.5f * z[e]);
+            dyv[e] = live ? scale * (fmaf(0.5f, th, 0.5f) - y) : 0.f;
+            lin += fmaxf(z[e], 0.f) - z[e] * y;
+            prod *= fmaf(0.5f, fabsf(th), 0.5f);
+          }
+          if (live) loss_acc += lin - __logf(prod);
+#pragma unroll
+          for (int hq = 0; hq < NC / 8; ++hq) {
+            const uint4 v = make_uint4(pack_bf16x2(dyv[8 * hq], dyv[8 * hq + 1]),
+                                       pack_bf16x2(dyv[8 * hq + 2], dyv[8 * hq + 3]),
+                                       pack_bf16x2(dyv[8 * hq + 4], dyv[8 * hq + 5]),
+                                       pack_bf16x2(dyv[8 * hq + 6], dyv[8 * hq + 7]));
+            const int col = hh * CH + c + 8 * hq;
+            *reinterpret_cast<uint4*>(dyrow + swz_rows((uint32_t)(b * RB + col * 2), RB)) = v;
+            if (live) *reinterpret_cast<uint4*>(dyg + (int64_t)b * kG + col) = v;
+          }
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&dy_full[s]);
+      if (!wait_or_abort(&dw_full[s], (i >> 1) & 1, abort_flag)) break;
+      tc_fence_after();
+      // dW readout: row = slot r, columns = this warp's labels
+#pragma unroll
+      for (int c = 0; c < CH; c += 16) {
+        constexpr int NC = CH < 16 ? CH : 16;
+        float v[16];
+        if constexpr (NC == 8) tmem_ld8(D(s) + lane_off + (uint32_t)(hh * CH + c), v);
+        else tmem_ld16(D(s) + lane_off + (uint32_t)(hh * CH + c), v);
+        tmem_wait_ld();
+        if (r < kK) {
+          __nv_bfloat16* dst = a.dW + (g * kG + hh * CH + c) * kK + r;
+#pragma unroll
+          for (int e = 0; e < NC; ++e) dst[(int64_t)e * kK] = __float2bfloat16_rn(v[e]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tmem_empty[s]);
+    }
+    // deterministic loss reduction over the 8 epilogue warps (named barrier 1)
+    float v = loss_acc;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (lane == 0) red[ew] = v;
+    named_bar(1, 256);
+    if (ew == 0 && lane == 0) {
+      float t = 0.f;
+      for (int j = 0; j < 8; ++j) t += red[j];
+      a.loss_part[blockIdx.x] = t;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (w == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem, ncols);
+  }
+}
+
+// ============================================================== k_dx2
+constexpr int kDxThreads = 672;  // 4 producer warps, MMA warp, 16 scatter warps
+
+template <int kG, int kK>
+__global__ void __launch_bounds__(kDxThreads, 1)
+    k_dx2(DxArgs a, const __nv_bfloat16* __restrict__ dY, const __nv_bfloat16* __restrict__ W) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  constexpr int RB = kG * 2;
+  constexpr int NS = dx_stages<kG>();
+  const TailShape sh = a.sh;
+  const int n_bt = sh.Bp / 128;
+  const int per_chunk = n_bt * a.n_bands;
+  const int c = blockIdx.x / per_chunk;
+  const int h = (blockIdx.x % per_chunk) / n_bt;
+  const int t = blockIdx.x % n_bt;
+  const int f0 = h * a.band;
+  const int f1 = min(sh.d, f0 + a.band);
+  const int64_t g0 = (int64_t)c * sh.n_groups / a.n_chunks;
+  const int64_t g1 = (int64_t)(c + 1) * sh.n_groups / a.n_chunks;
+
+  const DxLayout Lo = dx_layout(a.band, kK, kG, NS);
+  const uint32_t base = align1024(smem_u32(smem));
+  uint8_t* gbase = smem + (base - smem_u32(smem));
+  float* acc = reinterpret_cast<float*>(gbase + Lo.acc);
+  auto meta = [&](int ms) -> int32_t* { return reinterpret_cast<int32_t*>(gbase + Lo.meta + ms * Lo.meta_stride); };
+  auto DYS = [&](int ds) -> uint32_t { return base + Lo.dy + ds * Lo.dy_stride; };
+  auto WS = [&](int ds) -> uint32_t { return base + Lo.w + ds * Lo.w_stride; };
+  uint64_t* bars = reinterpret_cast<uint64_t*>(gbase + Lo.bars);
+  uint64_t* full = bars;                          // [NS] stage loaded (count: 128 producers)
+  uint64_t* empty = full + NS;                    // [NS] stage consumed by the MMA
+  uint64_t* meta_full = empty + NS;               // [8] metadata written (count: warp 0)
+  uint64_t* meta_empty = meta_full + kMetaSlots;  // [8] metadata consumed by the scatter
+  uint64_t* z_full = meta_empty + kMetaSlots;     // [2] Z in TMEM
+  uint64_t* tmem_empty = z_full + 2;              // [2] Z read out
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(tmem_empty + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
+
+  const int w = warp_id(), lane = lane_id();
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&full[s], 128);
+      mbar_init(&empty[s], 1);
+    }
+    for (int s = 0; s < kMetaSlots; ++s) {
+      mbar_init(&meta_full[s], 32);
+      mbar_init(&meta_empty[s], 16);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&z_full[s], 1);
+      mbar_init(&tmem_empty[s], 16);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  for (int i = threadIdx.x; i < a.band * 128; i += blockDim.x) acc[i] = 0.f;
+  constexpr uint32_t kZCols = 2 * kK <= 128 ? 128u : 256u;
+  if (w == 4) {
+    tmem_alloc(tslot, kZCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tslot;
+  auto Z = [&](int s) -> uint32_t { return tmem + (s ? (uint32_t)kK : 0u); };
+  // feature quarters of the band: [fq(j), fq(j+1)) belongs to scatter warps with p = j
+  auto fq = [&](int j) -> int { return min(f1, f0 + (a.band * j) / 4); };
+
+  if (w < 4) {
+    // ------------------------------------------------- cp.async producers
+    // Each producer warp reads the group's index row itself and derives the
+    // band's slot split points (idx is sorted); warp 0 also writes the metadata.
+    // A stage is published (proxy fence + arrive) NS-1 groups after its copies
+    // were issued, so NS stages are in flight.
+    const int tid = threadIdx.x;
+    int vals[kK / 32];
+    if (g0 < g1) {
+#pragma unroll
+      for (int j = 0; j < kK / 32; ++j) vals[j] = a.idx[g0 * kK + lane + 32 * j];
+    }
+    int i = 0;
+    bool stopped = false;
+    for (int64_t g = g0; g < g1; ++g) {
+      int cnt[5] = {0, 0, 0, 0, 0};
+      int cur[kK / 32];
+#pragma unroll
+      for (int j = 0; j < kK / 32; ++j) {
+        cur[j] = vals[j];
+#pragma unroll
+        for (int e = 0; e < 5; ++e) cnt[e] += __popc(__ballot_sync(0xffffffffu, cur[j] < fq(e)));
+      }
+      if (g + 1 < g1) {
+#pragma unroll
+        for (int j = 0; j < kK / 32; ++j) vals[j] = a.idx[(g + 1) * kK + lane + 32 * j];  // prefetch
+      }
+      const int lo = cnt[0], hi = cnt[4];
+      if (hi == lo) continue;  // no feature of this band in the group (uniform)
+      const int ds = i % NS, ms = i % kMetaSlots;
+      if (!wait_or_abort(&empty[ds], ((i / NS) & 1) ^ 1, abort_flag)) {
+        stopped = true;
+        break;
+      }
+      const int s0 = lo & ~63;
+      const int N = ((hi - s0 + 63) / 64) * 64;
+      if (w == 0) {
+        if (!wait_or_abort(&meta_empty[ms], ((i / kMetaSlots) & 1) ^ 1, abort_flag)) {
+          stopped = true;
+          break;
+        }
+        int32_t* m = meta(ms);
+#pragma unroll
+        for (int j = 0; j < kK / 32; ++j) {
+          const int sl = lane + 32 * j;
+          if (sl >= lo && sl < hi) m[kMetaHdr + sl - lo] = (cur[j] - f0) * 128;  // accumulator row offset
+        }
+        if (lane < 5) m[lane] = lane == 0 ? cnt[0] : lane == 1 ? cnt[1] : lane == 2 ? cnt[2] : lane == 3 ? cnt[3] : cnt[4];
+        if (lane == 0) {
+          m[5] = s0;
+          m[6] = N;
+        }
+        __syncwarp();
+        mbar_arrive(&meta_full[ms]);
+      }
+      // dY tile: 128 rows of G labels (rows at or beyond B read as zero)
+      const uint32_t dys = DYS(ds);
+      constexpr int cpr = kG / 8;
+      const __nv_bfloat16* dyg = dY + g * a.dy_gstride;
+#pragma unroll
+      for (int q0 = 0; q0 < 128 * cpr; q0 += 128) {
+        const int qq = q0 + tid;
+        const int b = qq / cpr, cc = qq % cpr;
+        const int row = t * 128 + b;
+        const bool in = row < sh.B;
+        cp_async16(dys + swz_rows((uint32_t)(b * RB + cc * 16), RB),
+                   in ? dyg + (int64_t)row * a.dy_rstride + cc * 8 : dY, in ? 16u : 0u);
+      }
+      // weight columns [s0, s0 + N) of the group's G x k block, 64-slot blocks
+      const uint32_t ws = WS(ds);
+      const __nv_bfloat16* wsrc = W + g * (int64_t)kG * kK + s0;
+      const int rowch = N / 8;
+      for (int qq = tid; qq < rowch * kG; qq += 128) {
+        const int j = qq / rowch, cc = qq % rowch;
+        cp_async16(ws + (uint32_t)((cc >> 3) * kG * 128) + sw128((uint32_t)(j * 128 + (cc & 7) * 16)),
+                   wsrc + (int64_t)j * kK + cc * 8, 16);
+      }
+      cp_async_commit();
+      if (i >= NS - 1) {
+        cp_async_wait_group<NS - 1>();
+        fence_proxy_async_smem();
+        mbar_arrive(&full[(i - (NS - 1)) % NS]);
+      }
+      ++i;
+    }
+    cp_async_wait_all();
+    if (!stopped) {
+      fence_proxy_async_smem();
+      for (int j = (i > NS - 1 ? i - (NS - 1) : 0); j < i; ++j) mbar_arrive(&full[j % NS]);
+      // end marker: metadata N = 0 and a data stage without copies
+      const int ds = i % NS, ms = i % kMetaSlots;
+      if (wait_or_abort(&empty[ds], ((i / NS) & 1) ^ 1, abort_flag)) {
+        if (w == 0 && wait_or_abort(&meta_empty[ms], ((i / kMetaSlots) & 1) ^ 1, abort_flag)) {
+          if (lane == 0) meta(ms)[6] = 0;
+          __syncwarp();
+          mbar_arrive(&meta_full[ms]);
+        }
+        named_bar(2, 128);
+        mbar_arrive(&full[ds]);
+      }
+    }
+  } else if (w == 4) {
+    // ------------------------------------------------------------- MMA
+    for (int i = 0;; ++i) {
+      const int ds = i % NS, ms = i % kMetaSlots;
+      if (!wait_or_abort(&full[ds], (i / NS) & 1, abort_flag)) break;
+      const int N = *reinterpret_cast<volatile int32_t*>(&meta(ms)[6]);
+      if (N == 0) break;
+      if (!wait_or_abort(&tmem_empty[i & 1], ((i >> 1) & 1) ^ 1, abort_flag)) break;
+      tc_fence_after();
+      if (lane == 0) {
+        const uint32_t idesc = make_idesc(1, 0, 1, 128, (uint32_t)N);
+        for (int kk = 0; kk < kG / 16; ++kk) {
+          const uint64_t ad = make_sdesc(DYS(ds) + (uint32_t)(kk * 32), 16, 8 * RB, layout_for_rows(RB));
+          const uint64_t bd = make_sdesc(WS(ds) + (uint32_t)(kk * 16 * 128), (uint32_t)kG * 128, 1024, kLayoutSw128);
+          mma_ss<false>(Z(i & 1), ad, bd, idesc, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&z_full[i & 1]);
+        mma_commit(&empty[ds]);
+      }
+      __syncwarp();
+    }
+  } else {
+    // ---------------------------------------------------------- scatter
+    const int q = w & 3, p = (w - 5) >> 2;  // batch quarter, feature quarter
+    const int b = q * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    for (int i = 0;; ++i) {
+      const int ms = i % kMetaSlots;
+      if (!wait_or_abort(&meta_full[ms], (i / kMetaSlots) & 1, abort_flag)) break;
+      const int32_t* m = meta(ms);
+      const int N = *reinterpret_cast<const volatile int32_t*>(&m[6]);
+      if (N == 0) break;
+      const int lo = m[0], beg = m[p], end = m[p + 1], s0 = m[5];
+      if (!wait_or_abort(&z_full[i & 1], (i >> 1) & 1, abort_flag)) break;
+      tc_fence_after();
+      for (int cc = (beg - s0) & ~15; cc < end - s0; cc += 16) {
+        float v[16], old[16];
+        int off[16];
+        tmem_ld16(Z(i & 1) + lane_off + (uint32_t)cc, v);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int sl = s0 + cc + e;
+          off[e] = (sl >= beg && sl < end) ? m[kMetaHdr + sl - lo] + b : -1;
+        }
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          if (off[e] >= 0) old[e] = acc[off[e]];
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          if (off[e] >= 0) acc[off[e]] = old[e] + v[e];
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&tmem_empty[i & 1]);
+        mbar_arrive(&meta_empty[ms]);
+      }
+    }
+    // this warp's features x batch columns -> chunk partial
+    for (int f = fq(p); f < fq(p + 1); ++f)
+      a.dX_part[((int64_t)c * sh.d + f) * sh.Bp + t * 128 + b] = acc[(f - f0) * 128 + b];
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (w == 4) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kZCols);
+  }
+}
+
+}  // namespace v2
+
+// ------------------------------------------------------------- host side
+namespace tail2 {
+
+bool supported(int G, int k, int Bp) {
+  return (G == 16 || G == 32 || G == 64) && (k == 64 || k == 128) && Bp <= 256;
+}
+
+size_t step_smem(int Bp, int k, int G) { return v2::step_layout(Bp, k, G).total; }
+size_t dx_smem(int band, int k, int G) {
+  return v2::dx_layout(band, k, G, G <= 32 ? v2::dx_stages<32>() : v2::dx_stages<64>()).total;
+}
+
+template <int kG, int kK>
+cudaError_t launch_step_t(const v2::StepArgs& a, int grid, const void* Xt, const void* W, cudaStream_t st) {
+  const size_t smem = step_smem(a.sh.Bp, kK, kG);
+  auto kern = v2::k_step2<kG, kK>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, v2::kStepThreads, smem, st>>>(a, static_cast<const __nv_bfloat16*>(Xt),
+                                             static_cast<const __nv_bfloat16*>(W));
+  return cudaGetLastError();
+}
+
+template <int kG, int kK>
+cudaError_t launch_dx_t(const v2::DxArgs& a, const void* dY, const void* W, cudaStream_t st) {
+  const size_t smem = dx_smem(a.band, kK, kG);
+  auto kern = v2::k_dx2<kG, kK>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const int grid = (a.sh.Bp / 128) * a.n_bands * a.n_chunks;
+  kern<<<grid, v2::kDxThreads, smem, st>>>(a, static_cast<const __nv_bfloat16*>(dY),
+                                           static_cast<const __nv_bfloat16*>(W));
+  return cudaGetLastError();
+}
+
+#define HASTE_V2_DISPATCH(FN, ...)                                     \
+  switch (G * 1000 + k) {                                              \
+    case 16064: return FN<16, 64>(__VA_ARGS__);                        \
+    case 16128: return FN<16, 128>(__VA_ARGS__);                       \
+    case 32064: return FN<32, 64>(__VA_ARGS__);                        \
+    case 32128: return FN<32, 128>(__VA_ARGS__);                       \
+    case 64064: return FN<64, 64>(__VA_ARGS__);                        \
+    case 64128: return FN<64, 128>(__VA_ARGS__);                       \
+    default: return cudaErrorInvalidValue;                             \
+  }
+
+cudaError_t launch_step(int G, int k, const v2::StepArgs& a, int grid, const void* Xt, const void* W,
+                        cudaStream_t st) {
+  HASTE_V2_DISPATCH(launch_step_t, a, grid, Xt, W, st)
+}
+
+cudaError_t launch_dx(int G, int k, const v2::DxArgs& a, const void* dY, const void* W, cudaStream_t st) {
+  HASTE_V2_DISPATCH(launch_dx_t, a, dY, W, st)
+}
+
+}  // namespace tail2
+}  // namespace haste
