@@ -122,9 +122,10 @@ class ProfScope {
 };
 
 // Tiling of the dX pass: feature bands sized so the fp32 band accumulator fits
-// next to the W and dY tiles; group chunks so that all CTAs are resident.
+// in shared memory next to the W and dY tiles (ns stages of them in the
+// pipelined kernel); group chunks so that all CTAs are resident.
 struct DxTiling {
-  int band, n_bands, n_chunks;
+  int band, n_bands, n_chunks, ns;
 };
 
 // The warp-specialised TMA kernels cover bf16 with G in {16, 32, 64}, k in
@@ -134,9 +135,14 @@ bool use_v2(const haste_plan_s& p, int Bp, int elem) { return elem == 2 && tail2
 
 DxTiling dx_tiling(const haste_plan_s& p, int Bp, int elem, int sms, int smem_optin) {
   DxTiling t{};
-  const size_t fixed = use_v2(p, Bp, elem) ? tail2::dx_smem(0, p.k, p.G) : tail::smem_dx(elem, p.k, p.G, 0);
-  long avail = (long)smem_optin - (long)fixed - 4096;  // headroom for static shared memory
-  int band = (int)std::min<long>(use_v2(p, Bp, elem) ? 512 : 256, avail / 512);
+  const int kHeadroom = 4096;  // static shared memory and launch reserve
+  int band = 8;
+  if (use_v2(p, Bp, elem)) {
+    if (!tail2::dx_config(p.G, p.k, p.d, (size_t)smem_optin, kHeadroom, &band, &t.ns)) t.ns = 2;
+  } else {
+    const long avail = (long)smem_optin - (long)tail::smem_dx(elem, p.k, p.G, 0) - kHeadroom;
+    band = (int)std::min<long>(256, avail / 512);
+  }
   band = std::max(8, band & ~7);
   if (band > p.d) band = round_up(p.d, 8);
   // as few bands as fit, then split d evenly between them
@@ -223,6 +229,7 @@ cudaError_t dx_v2(const haste_plan_s& p, int B, const void* W, const void* dY, i
   a.band = t.band;
   a.n_bands = t.n_bands;
   a.n_chunks = t.n_chunks;
+  a.ns = t.ns;
   a.dy_gstride = gstride;
   a.dy_rstride = rstride;
   return tail2::launch_dx(p.G, p.k, a, dY, W, s);

@@ -13,11 +13,12 @@
 //              buffer of the dX pass), then dW is read out of TMEM.
 // k_dx2 -- dX pass: per CTA (128-row batch tile, feature band, group chunk):
 //   warps 0-3 stage the dY tile and the weight columns of the band's slots
-//   (multi-stage ring; warp 0 also writes the slot metadata into an 8-entry ring),
+//   (multi-stage ring; warp 0 also writes the slot metadata into a 16-entry ring),
 //   warp 4 issues Z = dY_g . W_g[:, slots], warps 5-20 add the rows of Z into a
-//   fp32 band accumulator in shared memory.  Scatter warp (q, p) owns batch rows
-//   [32q, 32q+32) and the p-th quarter of the band's features, so every feature
-//   receives its group terms in ascending group order, deterministically.
+//   fp32 band accumulator held in TMEM (lane = batch row, column = feature).
+//   Scatter warp (q, p) owns batch rows [32q, 32q+32) and the p-th quarter of the
+//   band's features, so every feature receives its group terms in ascending
+//   group order, deterministically.
 #include "tail.cuh"
 
 namespace haste {
@@ -38,18 +39,15 @@ struct DxArgs {
   TailShape sh;
   const int32_t* idx;
   float* dX_part;
-  int band, n_bands, n_chunks;
+  int band, n_bands, n_chunks, ns;  // ns: stages of the shared-memory ring
   // element (b, g*G + j) of dY is at dY[g*dy_gstride + b*dy_rstride + j]
   int64_t dy_gstride, dy_rstride;
 };
 
-constexpr int kMetaSlots = 8;  // metadata ring of the dX pass
+constexpr int kMetaSlots = 16;  // metadata ring of the dX pass (twice the deepest data ring)
 constexpr int kMetaHdr = 8;    // 5 slot split points, s0, N, 1 spare
 
-template <int kG>
-__host__ __device__ constexpr int dx_stages() {
-  return kG <= 32 ? 4 : 3;
-}
+constexpr int kMaxDxStages = 8;  // deepest data ring of the dX pass
 
 // ------------------------------------------------------------ smem layouts
 struct StepLayout {
@@ -73,6 +71,8 @@ __host__ __device__ inline StepLayout step_layout(int Bp, int k, int G) {
 struct DxLayout {
   uint32_t dy, w, acc, meta, bars, total, dy_stride, w_stride, meta_stride;
 };
+// Shared memory of the dX pass: ns stages of (dY tile, weight columns), the fp32
+// band accumulator [band][128], the metadata ring and the barriers.
 __host__ __device__ inline DxLayout dx_layout(int band, int k, int G, int ns) {
   DxLayout L;
   L.dy_stride = (uint32_t)((128 * G * 2 + 1023) & ~1023);
@@ -379,13 +379,27 @@ __global__ void __launch_bounds__(kStepThreads, 1)
 
 // ============================================================== k_dx2
 constexpr int kDxThreads = 672;  // 4 producer warps, MMA warp, 16 scatter warps
+constexpr int kZBufs = 4;        // Z buffers in TMEM (kK columns each)
 
+// One CTA owns a band [f0, f1) of input features for a 128-row batch tile and a
+// chunk of groups.  For each group that has slots in the band:
+//   producers (warps 0-3): dY tile (128 x G) and the weight columns of the band's
+//     slots into a stage of the shared-memory ring (cp.async, completion tracked
+//     by the stage's mbarrier); warp 0 writes the slot -> accumulator-column map;
+//   MMA (warp 4): Z = dY_g W_g[:, slots] (128 x N, fp32) into one of four TMEM
+//     buffers;
+//   scatter (warps 5-20): each warp owns 32 batch rows x a quarter of the band and
+//     adds its Z columns into the fp32 band accumulator in shared memory.
+// Feature ownership is fixed per warp, so warps on different groups never touch
+// the same accumulator element; the slot order within a group is the index
+// order, so each accumulator element sums its terms in group order.
 template <int kG, int kK>
 __global__ void __launch_bounds__(kDxThreads, 1)
     k_dx2(DxArgs a, const __nv_bfloat16* __restrict__ dY, const __nv_bfloat16* __restrict__ W) {
   extern __shared__ __align__(1024) uint8_t smem[];
   constexpr int RB = kG * 2;
-  constexpr int NS = dx_stages<kG>();
+  constexpr int kPf = kK / 32;  // index registers per lane for one group row
+  const int NS = a.ns;
   const TailShape sh = a.sh;
   const int n_bt = sh.Bp / 128;
   const int per_chunk = n_bt * a.n_bands;
@@ -400,18 +414,18 @@ __global__ void __launch_bounds__(kDxThreads, 1)
   const DxLayout Lo = dx_layout(a.band, kK, kG, NS);
   const uint32_t base = align1024(smem_u32(smem));
   uint8_t* gbase = smem + (base - smem_u32(smem));
-  float* acc = reinterpret_cast<float*>(gbase + Lo.acc);
+  float* acc = reinterpret_cast<float*>(gbase + Lo.acc);  // [band][128] fp32
   auto meta = [&](int ms) -> int32_t* { return reinterpret_cast<int32_t*>(gbase + Lo.meta + ms * Lo.meta_stride); };
   auto DYS = [&](int ds) -> uint32_t { return base + Lo.dy + ds * Lo.dy_stride; };
   auto WS = [&](int ds) -> uint32_t { return base + Lo.w + ds * Lo.w_stride; };
   uint64_t* bars = reinterpret_cast<uint64_t*>(gbase + Lo.bars);
-  uint64_t* full = bars;                          // [NS] stage loaded (count: 128 producers)
-  uint64_t* empty = full + NS;                    // [NS] stage consumed by the MMA
-  uint64_t* meta_full = empty + NS;               // [8] metadata written (count: warp 0)
-  uint64_t* meta_empty = meta_full + kMetaSlots;  // [8] metadata consumed by the scatter
-  uint64_t* z_full = meta_empty + kMetaSlots;     // [2] Z in TMEM
-  uint64_t* tmem_empty = z_full + 2;              // [2] Z read out
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(tmem_empty + 2);
+  uint64_t* full = bars;                          // [NS] stage landed (count: 128 producer threads)
+  uint64_t* empty = full + kMaxDxStages;          // [NS] stage consumed by the MMA
+  uint64_t* meta_full = empty + kMaxDxStages;     // [16] metadata written (count: warp 0)
+  uint64_t* meta_empty = meta_full + kMetaSlots;  // [16] metadata consumed by the scatter
+  uint64_t* z_full = meta_empty + kMetaSlots;     // [4] Z in TMEM
+  uint64_t* z_empty = z_full + kZBufs;            // [4] Z read out
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(z_empty + kZBufs);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
 
   const int w = warp_id(), lane = lane_id();
@@ -424,82 +438,79 @@ __global__ void __launch_bounds__(kDxThreads, 1)
       mbar_init(&meta_full[s], 32);
       mbar_init(&meta_empty[s], 16);
     }
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kZBufs; ++s) {
       mbar_init(&z_full[s], 1);
-      mbar_init(&tmem_empty[s], 16);
+      mbar_init(&z_empty[s], 16);
     }
     *abort_flag = 0;
     fence_mbar_init();
   }
-  for (int i = threadIdx.x; i < a.band * 128; i += blockDim.x) acc[i] = 0.f;
-  constexpr uint32_t kZCols = 2 * kK <= 128 ? 128u : 256u;
+  constexpr uint32_t kTmemCols = kZBufs * kK;
   if (w == 4) {
-    tmem_alloc(tslot, kZCols);
+    tmem_alloc(tslot, kTmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tslot;
-  auto Z = [&](int s) -> uint32_t { return tmem + (s ? (uint32_t)kK : 0u); };
+  auto Z = [&](int s) -> uint32_t { return tmem + (uint32_t)(s * kK); };
   // feature quarters of the band: [fq(j), fq(j+1)) belongs to scatter warps with p = j
   auto fq = [&](int j) -> int { return min(f1, f0 + (a.band * j) / 4); };
 
   if (w < 4) {
     // ------------------------------------------------- cp.async producers
-    // Each producer warp reads the group's index row itself and derives the
-    // band's slot split points (idx is sorted); warp 0 also writes the metadata.
-    // A stage is published (proxy fence + arrive) NS-1 groups after its copies
-    // were issued, so NS stages are in flight.
+    // Each producer warp reads the group's index row itself (two rows ahead) and
+    // derives the band's slot split points (idx is sorted); warp 0 also writes
+    // the metadata.  Each thread's copies of a stage arrive on the stage's full
+    // barrier when they land, so up to NS stages are in flight.
     const int tid = threadIdx.x;
-    int vals[kK / 32];
-    if (g0 < g1) {
+    int va[kPf], vb[kPf];  // index rows of groups g (even offset) and g + 1 (odd offset)
 #pragma unroll
-      for (int j = 0; j < kK / 32; ++j) vals[j] = a.idx[g0 * kK + lane + 32 * j];
+    for (int j = 0; j < kPf; ++j) {
+      va[j] = g0 < g1 ? a.idx[g0 * kK + lane + 32 * j] : 0;
+      vb[j] = g0 + 1 < g1 ? a.idx[(g0 + 1) * kK + lane + 32 * j] : 0;
     }
-    int i = 0;
+    int i = 0, ds = 0, dph = 0;
     bool stopped = false;
-    for (int64_t g = g0; g < g1; ++g) {
+    // One group: v holds its index row on entry and the row of g + 2 on exit (the
+    // load is only consumed two groups later, so its latency stays hidden).
+    auto produce = [&](int64_t g, int (&v)[kPf]) -> bool {
       int cnt[5] = {0, 0, 0, 0, 0};
-      int cur[kK / 32];
 #pragma unroll
-      for (int j = 0; j < kK / 32; ++j) {
-        cur[j] = vals[j];
+      for (int j = 0; j < kPf; ++j) {
 #pragma unroll
-        for (int e = 0; e < 5; ++e) cnt[e] += __popc(__ballot_sync(0xffffffffu, cur[j] < fq(e)));
-      }
-      if (g + 1 < g1) {
-#pragma unroll
-        for (int j = 0; j < kK / 32; ++j) vals[j] = a.idx[(g + 1) * kK + lane + 32 * j];  // prefetch
+        for (int e = 0; e < 5; ++e) cnt[e] += __popc(__ballot_sync(0xffffffffu, v[j] < fq(e)));
       }
       const int lo = cnt[0], hi = cnt[4];
-      if (hi == lo) continue;  // no feature of this band in the group (uniform)
-      const int ds = i % NS, ms = i % kMetaSlots;
-      if (!wait_or_abort(&empty[ds], ((i / NS) & 1) ^ 1, abort_flag)) {
-        stopped = true;
-        break;
-      }
-      const int s0 = lo & ~63;
-      const int N = ((hi - s0 + 63) / 64) * 64;
-      if (w == 0) {
-        if (!wait_or_abort(&meta_empty[ms], ((i / kMetaSlots) & 1) ^ 1, abort_flag)) {
-          stopped = true;
-          break;
-        }
+      const int ms = i % kMetaSlots;
+      if (hi > lo && w == 0) {
+        if (!wait_or_abort(&meta_empty[ms], ((i / kMetaSlots) & 1) ^ 1, abort_flag)) return false;
         int32_t* m = meta(ms);
 #pragma unroll
-        for (int j = 0; j < kK / 32; ++j) {
+        for (int j = 0; j < kPf; ++j) {
           const int sl = lane + 32 * j;
-          if (sl >= lo && sl < hi) m[kMetaHdr + sl - lo] = (cur[j] - f0) * 128;  // accumulator row offset
+          if (sl >= lo && sl < hi) m[kMetaHdr + sl - lo] = (v[j] - f0) * 128;  // accumulator row offset
         }
+      }
+      if (g + 2 < g1) {
+#pragma unroll
+        for (int j = 0; j < kPf; ++j) v[j] = a.idx[(g + 2) * kK + lane + 32 * j];  // prefetch
+      }
+      if (hi == lo) return true;  // no feature of this band in the group (uniform)
+      const int s0 = lo & ~63;
+      const int nblk = (hi - s0 + 63) / 64;  // 64-slot blocks of weight columns
+      if (w == 0) {
+        int32_t* m = meta(ms);
         if (lane < 5) m[lane] = lane == 0 ? cnt[0] : lane == 1 ? cnt[1] : lane == 2 ? cnt[2] : lane == 3 ? cnt[3] : cnt[4];
         if (lane == 0) {
           m[5] = s0;
-          m[6] = N;
+          m[6] = nblk * 64;
         }
         __syncwarp();
         mbar_arrive(&meta_full[ms]);
       }
+      if (!wait_or_abort(&empty[ds], dph ^ 1, abort_flag)) return false;
       // dY tile: 128 rows of G labels (rows at or beyond B read as zero)
       const uint32_t dys = DYS(ds);
       constexpr int cpr = kG / 8;
@@ -513,107 +524,140 @@ __global__ void __launch_bounds__(kDxThreads, 1)
         cp_async16(dys + swz_rows((uint32_t)(b * RB + cc * 16), RB),
                    in ? dyg + (int64_t)row * a.dy_rstride + cc * 8 : dY, in ? 16u : 0u);
       }
-      // weight columns [s0, s0 + N) of the group's G x k block, 64-slot blocks
+      // weight columns [s0, s0 + 64*nblk) of the group's G x k block
       const uint32_t ws = WS(ds);
       const __nv_bfloat16* wsrc = W + g * (int64_t)kG * kK + s0;
-      const int rowch = N / 8;
-      for (int qq = tid; qq < rowch * kG; qq += 128) {
-        const int j = qq / rowch, cc = qq % rowch;
-        cp_async16(ws + (uint32_t)((cc >> 3) * kG * 128) + sw128((uint32_t)(j * 128 + (cc & 7) * 16)),
-                   wsrc + (int64_t)j * kK + cc * 8, 16);
+      for (int blk = 0; blk < nblk; ++blk) {
+#pragma unroll
+        for (int r = 0; r < kG / 16; ++r) {
+          const int qq = tid + 128 * r;
+          const int j = qq >> 3, cc = qq & 7;
+          cp_async16(ws + (uint32_t)(blk * kG * 128) + sw128((uint32_t)(j * 128 + cc * 16)),
+                     wsrc + (int64_t)j * kK + blk * 64 + cc * 8, 16);
+        }
       }
-      cp_async_commit();
-      if (i >= NS - 1) {
-        cp_async_wait_group<NS - 1>();
-        fence_proxy_async_smem();
-        mbar_arrive(&full[(i - (NS - 1)) % NS]);
-      }
+      cp_async_arrive_on(&full[ds]);  // the stage publishes itself when its copies land
       ++i;
+      if (++ds == NS) {
+        ds = 0;
+        dph ^= 1;
+      }
+      return true;
+    };
+    for (int64_t g = g0; g < g1; g += 2) {
+      if (!produce(g, va) || (g + 1 < g1 && !produce(g + 1, vb))) {
+        stopped = true;
+        break;
+      }
     }
     cp_async_wait_all();
     if (!stopped) {
-      fence_proxy_async_smem();
-      for (int j = (i > NS - 1 ? i - (NS - 1) : 0); j < i; ++j) mbar_arrive(&full[j % NS]);
       // end marker: metadata N = 0 and a data stage without copies
-      const int ds = i % NS, ms = i % kMetaSlots;
-      if (wait_or_abort(&empty[ds], ((i / NS) & 1) ^ 1, abort_flag)) {
+      const int ms = i % kMetaSlots;
+      if (wait_or_abort(&empty[ds], dph ^ 1, abort_flag)) {
         if (w == 0 && wait_or_abort(&meta_empty[ms], ((i / kMetaSlots) & 1) ^ 1, abort_flag)) {
           if (lane == 0) meta(ms)[6] = 0;
           __syncwarp();
           mbar_arrive(&meta_full[ms]);
         }
-        named_bar(2, 128);
         mbar_arrive(&full[ds]);
       }
     }
   } else if (w == 4) {
     // ------------------------------------------------------------- MMA
+    int ds = 0, dph = 0;
     for (int i = 0;; ++i) {
-      const int ds = i % NS, ms = i % kMetaSlots;
-      if (!wait_or_abort(&full[ds], (i / NS) & 1, abort_flag)) break;
+      const int ms = i % kMetaSlots, zs = i % kZBufs;
+      if (!wait_or_abort(&full[ds], dph, abort_flag)) break;
+      if (!wait_or_abort(&meta_full[ms], (i / kMetaSlots) & 1, abort_flag)) break;
+      fence_proxy_async_smem();  // landed cp.async data is read by the tensor core
       const int N = *reinterpret_cast<volatile int32_t*>(&meta(ms)[6]);
       if (N == 0) break;
-      if (!wait_or_abort(&tmem_empty[i & 1], ((i >> 1) & 1) ^ 1, abort_flag)) break;
+      if (!wait_or_abort(&z_empty[zs], ((i / kZBufs) & 1) ^ 1, abort_flag)) break;
       tc_fence_after();
       if (lane == 0) {
         const uint32_t idesc = make_idesc(1, 0, 1, 128, (uint32_t)N);
         for (int kk = 0; kk < kG / 16; ++kk) {
           const uint64_t ad = make_sdesc(DYS(ds) + (uint32_t)(kk * 32), 16, 8 * RB, layout_for_rows(RB));
           const uint64_t bd = make_sdesc(WS(ds) + (uint32_t)(kk * 16 * 128), (uint32_t)kG * 128, 1024, kLayoutSw128);
-          mma_ss<false>(Z(i & 1), ad, bd, idesc, kk > 0 ? 1u : 0u);
+          mma_ss<false>(Z(zs), ad, bd, idesc, kk > 0 ? 1u : 0u);
         }
-        mma_commit(&z_full[i & 1]);
+        mma_commit(&z_full[zs]);
         mma_commit(&empty[ds]);
       }
       __syncwarp();
+      if (++ds == NS) {
+        ds = 0;
+        dph ^= 1;
+      }
     }
   } else {
     // ---------------------------------------------------------- scatter
     const int q = w & 3, p = (w - 5) >> 2;  // batch quarter, feature quarter
     const int b = q * 32 + lane;
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    float* accb = acc + b;
+    for (int f = fq(p); f < fq(p + 1); ++f) accb[(f - f0) * 128] = 0.f;
     for (int i = 0;; ++i) {
-      const int ms = i % kMetaSlots;
+      const int ms = i % kMetaSlots, zs = i % kZBufs;
       if (!wait_or_abort(&meta_full[ms], (i / kMetaSlots) & 1, abort_flag)) break;
       const int32_t* m = meta(ms);
       const int N = *reinterpret_cast<const volatile int32_t*>(&m[6]);
       if (N == 0) break;
       const int lo = m[0], beg = m[p], end = m[p + 1], s0 = m[5];
-      if (!wait_or_abort(&z_full[i & 1], (i >> 1) & 1, abort_flag)) break;
+      const int32_t* mo = m + kMetaHdr - lo;  // accumulator row offset of slot sl: mo[sl]
+      // Every warp waits for Z before it releases the buffer, also without slots
+      // in this group: a release may only count toward this group's phase.
+      if (!wait_or_abort(&z_full[zs], (i / kZBufs) & 1, abort_flag)) break;
       tc_fence_after();
-      for (int cc = (beg - s0) & ~15; cc < end - s0; cc += 16) {
-        float v[16], old[16];
-        int off[16];
-        tmem_ld16(Z(i & 1) + lane_off + (uint32_t)cc, v);
+      const uint32_t zcol = Z(zs) + lane_off - (uint32_t)s0;  // TMEM address of slot sl: zcol + sl
+      auto release_z = [&]() {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&z_empty[zs]);
+      };
+      int sl = beg;
+      if (sl >= end) release_z();
+      for (; sl + 8 <= end; sl += 8) {  // full batches of 8 slots
+        float v[8];
+        int off[8];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int sl = s0 + cc + e;
-          off[e] = (sl >= beg && sl < end) ? m[kMetaHdr + sl - lo] + b : -1;
-        }
+        for (int e = 0; e < 8; ++e) v[e] = tmem_ld1(zcol + (uint32_t)(sl + e));
+#pragma unroll
+        for (int e = 0; e < 8; ++e) off[e] = mo[sl + e];
         tmem_wait_ld();
+        if (sl + 8 == end) release_z();
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
-          if (off[e] >= 0) old[e] = acc[off[e]];
-#pragma unroll
-        for (int e = 0; e < 16; ++e)
-          if (off[e] >= 0) acc[off[e]] = old[e] + v[e];
+        for (int e = 0; e < 8; ++e) accb[off[e]] += v[e];
       }
-      tc_fence_before();
+      if (sl < end) {  // the last 1..7 slots (warp-uniform branches)
+        const int n = end - sl;
+        float v[7];
+        int off[7];
+#pragma unroll
+        for (int e = 0; e < 7; ++e)
+          if (e < n) v[e] = tmem_ld1(zcol + (uint32_t)(sl + e));
+#pragma unroll
+        for (int e = 0; e < 7; ++e)
+          if (e < n) off[e] = mo[sl + e];
+        tmem_wait_ld();
+        release_z();
+#pragma unroll
+        for (int e = 0; e < 7; ++e)
+          if (e < n) accb[off[e]] += v[e];
+      }
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&tmem_empty[i & 1]);
-        mbar_arrive(&meta_empty[ms]);
-      }
+      if (lane == 0) mbar_arrive(&meta_empty[ms]);
     }
-    // this warp's features x batch columns -> chunk partial
+    // this warp's features x batch rows -> chunk partial
     for (int f = fq(p); f < fq(p + 1); ++f)
-      a.dX_part[((int64_t)c * sh.d + f) * sh.Bp + t * 128 + b] = acc[(f - f0) * 128 + b];
+      a.dX_part[((int64_t)c * sh.d + f) * sh.Bp + t * 128 + b] = accb[(f - f0) * 128];
   }
   tc_fence_before();
   __syncthreads();
   if (w == 4) {
     tc_fence_after();
-    tmem_dealloc(tmem, kZCols);
+    tmem_dealloc(tmem, kTmemCols);
   }
 }
 
@@ -627,8 +671,25 @@ bool supported(int G, int k, int Bp) {
 }
 
 size_t step_smem(int Bp, int k, int G) { return v2::step_layout(Bp, k, G).total; }
-size_t dx_smem(int band, int k, int G) {
-  return v2::dx_layout(band, k, G, G <= 32 ? v2::dx_stages<32>() : v2::dx_stages<64>()).total;
+size_t dx_smem(int band, int k, int G, int ns) { return v2::dx_layout(band, k, G, ns).total; }
+
+// Band width and ring depth of the dX pass: the fewest bands whose accumulator
+// still leaves at least three stages (up to eight) in the shared memory left
+// after `reserve` bytes.  Returns false when even a band of 8 features does not fit.
+bool dx_config(int G, int k, int d, size_t smem_optin, size_t reserve, int* band, int* ns) {
+  const v2::DxLayout one = v2::dx_layout(0, k, G, 1), none = v2::dx_layout(0, k, G, 0);
+  const long stage = (long)one.total - (long)none.total;
+  for (int nb = 1; nb <= (d + 7) / 8; ++nb) {
+    const int bw = ((d + nb - 1) / nb + 7) & ~7;
+    const long left = (long)smem_optin - (long)reserve - (long)dx_smem(bw, k, G, 0);
+    const long n = left / stage;
+    if (n >= 3 || (bw == 8 && n >= 2)) {
+      *band = bw;
+      *ns = (int)std::min<long>(n, v2::kMaxDxStages);
+      return true;
+    }
+  }
+  return false;
 }
 
 template <int kG, int kK>
@@ -644,7 +705,7 @@ cudaError_t launch_step_t(const v2::StepArgs& a, int grid, const void* Xt, const
 
 template <int kG, int kK>
 cudaError_t launch_dx_t(const v2::DxArgs& a, const void* dY, const void* W, cudaStream_t st) {
-  const size_t smem = dx_smem(a.band, kK, kG);
+  const size_t smem = dx_smem(a.band, kK, kG, a.ns);
   auto kern = v2::k_dx2<kG, kK>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
