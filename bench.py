@@ -226,6 +226,20 @@ class Runner:
         self.h_out.copy_(src, non_blocking=True)
 
 
+def max_over_ranks(ms, device):
+    """The slowest rank's time: every rank contributes its own device-timed ms."""
+    import torch
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(world, batch, steps, ms):
+    """Whole-job throughput: every rank runs its own replica on its own batch of
+    `batch` samples (weak scaling), the job takes the slowest rank's time."""
+    return world * batch * steps / (ms / 1e3)
+
+
 def timed(fn, steps, warmup, dist):
     import torch
     for _ in range(warmup):
@@ -244,9 +258,7 @@ def timed(fn, steps, warmup, dist):
         torch.distributed.barrier()
     ms = e0.elapsed_time(e1)
     if dist:
-        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+        ms = max_over_ranks(ms, "cuda")
     return ms
 
 
@@ -402,7 +414,7 @@ def main():
     tail_ms = sum(prof[k][1] for k in prof if k.startswith("tail") or k in ("xt", "dx_reduce")) / args.steps
     tail_rf = roofline_of(work["tail"][0], work["tail"][1], tail_ms, peaks)
 
-    value = world * wl.B * args.steps / (ms / 1e3)
+    value = job_value(world, wl.B, args.steps, ms)
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 4), "higher_is_better": True,
@@ -414,7 +426,7 @@ def main():
                  "roofline": tail_rf},
         "kernels": {k: {"launches": n, "ms_per_launch": round(t / n, 4), "share": round(t / sum(
             x[1] for x in prof.values()), 4)} for k, (n, t) in prof.items()},
-        "e2e": {"value": round(world * wl.B * args.steps / (ms_e2e / 1e3), 1), "unit": UNIT,
+        "e2e": {"value": round(job_value(world, wl.B, args.steps, ms_e2e), 1), "unit": UNIT,
                 "h2d_bytes_per_step": run.h2d, "d2h_bytes_per_step": run.d2h},
         "gpu_launches": launches,
         "clocks": clocks,

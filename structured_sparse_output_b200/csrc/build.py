@@ -10,8 +10,10 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 PKG = os.path.dirname(HERE)
 OUT = os.path.join(PKG, "libhaste.so")
-SOURCES = ["api.cu", "tail.cu", "head.cu", "common.cuh", "tail.cuh",
-           os.path.join("..", "..", "include", "haste.h")]
+def _sources():
+    """Every CUDA source and header of the library, and the ABI header."""
+    own = [f for f in os.listdir(HERE) if f.endswith((".cu", ".cuh"))]
+    return own + [os.path.join("..", "..", "include", "haste.h")]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",
          "--expt-relaxed-constexpr", "-maxrregcount=152", "-Xcompiler", "-fPIC,-O2", "-shared"]
@@ -21,7 +23,7 @@ def stale() -> bool:
     if not os.path.exists(OUT):
         return True
     t = os.path.getmtime(OUT)
-    return any(os.path.getmtime(os.path.join(HERE, s)) > t for s in SOURCES)
+    return any(os.path.getmtime(os.path.join(HERE, s)) > t for s in _sources())
 
 
 def build(force: bool = False, verbose: bool = False) -> str:

@@ -3,19 +3,20 @@
 // Methodology 1: labels in groups of G share one fan-in set I_g of k features).
 //
 // k_step2 -- fused forward + BCE gradient + dW, one group per iteration:
-//   warps 0-1  producers: the gather-once tile X[:, I_g] (k rows of X^T) and the
-//              G x k weight block, staged with cp.async into a 2-stage ring; warp
-//              0 owns stage 0 and warp 1 stage 1;
-//   warp 2     MMA issuer (one thread): forward of group i+1 is issued before the
+//   warps 0-3  producers: the gather-once tile X[:, I_g] (k rows of X^T) and the
+//              G x k weight block, staged with cp.async into a 2-stage ring; warps
+//              0 and 2 fill stage 0, warps 1 and 3 stage 1;
+//   warp 4     MMA issuer (one thread): forward of group i+1 is issued before the
 //              dW of group i, so the tensor core works while the epilogue runs;
-//   warps 3-10 epilogue: logits leave TMEM only as the BCE gradient (bf16, to
+//   warps 5-12 epilogue: logits leave TMEM only as the BCE gradient (bf16, to
 //              shared memory for the dW product and to the group-major gradient
 //              buffer of the dX pass), then dW is read out of TMEM.
 // k_dx2 -- dX pass: per CTA (128-row batch tile, feature band, group chunk):
-//   warps 0-3 stage the dY tile and the weight columns of the band's slots
-//   (multi-stage ring; warp 0 also writes the slot metadata into a 16-entry ring),
-//   warp 4 issues Z = dY_g . W_g[:, slots], warps 5-20 add the rows of Z into a
-//   fp32 band accumulator held in TMEM (lane = batch row, column = feature).
+//   warps 0-3 stage the dY tile and the weight columns of the band's slots into
+//   a shared-memory ring whose stages publish themselves when their copies land
+//   (warp 0 also writes the slot metadata into a 16-entry ring), warp 4 issues
+//   Z = dY_g . W_g[:, slots] into one of four TMEM buffers, warps 5-20 add the
+//   columns of Z into a fp32 band accumulator in shared memory.
 //   Scatter warp (q, p) owns batch rows [32q, 32q+32) and the p-th quarter of the
 //   band's features, so every feature receives its group terms in ascending
 //   group order, deterministically.
@@ -76,6 +77,9 @@ struct DxLayout {
 __host__ __device__ inline DxLayout dx_layout(int band, int k, int G, int ns) {
   DxLayout L;
   L.dy_stride = (uint32_t)((128 * G * 2 + 1023) & ~1023);
+  // 64-slot blocks of weight columns: rows [s0, hi) of Z^T need two blocks only
+  // when k = 128 (hi - s0 <= k); with k = 64 the second block the MMA reads is the
+  // next region of shared memory and feeds only TMEM lanes no thread reads.
   L.w_stride = (uint32_t)((k / 64) * G * 128);
   L.meta_stride = (uint32_t)(kMetaHdr + k) * 4;
   uint32_t off = 0;
@@ -116,7 +120,9 @@ __device__ __forceinline__ void publish_all(uint64_t* full_bar) {
 }
 
 // ============================================================ k_step2
-constexpr int kStepThreads = 352;  // 2 producer warps, MMA warp, 8 epilogue warps (<= 3 per scheduler)
+constexpr int kStepProd = 4;       // producer warps: two per ring stage
+constexpr int kStepMma = kStepProd;  // warp id of the MMA issuer
+constexpr int kStepThreads = 32 * (kStepProd + 1 + 8);  // producers, MMA warp, 8 epilogue warps
 constexpr int kMaxPosReg = 8;      // positives per batch row kept in registers
 
 template <int kG, int kK>
@@ -145,7 +151,7 @@ __global__ void __launch_bounds__(kStepThreads, 1)
   const int w = warp_id(), lane = lane_id();
   if (threadIdx.x == 0) {
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&full[s], 32);
+      mbar_init(&full[s], 32 * kStepProd / 2);
       mbar_init(&empty[s], 1);
       mbar_init(&fwd_full[s], 1);
       mbar_init(&dy_full[s], 8);
@@ -158,7 +164,7 @@ __global__ void __launch_bounds__(kStepThreads, 1)
   // TMEM: forward accumulators F[2] (n_bt*G columns each), dW accumulators D[2]
   const uint32_t f_cols = (uint32_t)(n_bt * kG);
   const uint32_t ncols = tmem_cols_for(2 * f_cols + 2 * kG);
-  if (w == 2) {
+  if (w == kStepMma) {
     tmem_alloc(tslot, ncols);
     tmem_relinquish();
   }
@@ -177,38 +183,41 @@ __global__ void __launch_bounds__(kStepThreads, 1)
   const int64_t ge = (int64_t)(blockIdx.x + 1) * sh.n_groups / gridDim.x;
   const int n_items = (int)(ge - gb);
 
-  if (w < 2) {
+  if (w < kStepProd) {
     // ------------------------------------------------- cp.async producers
-    // warp h fills stage h with the items i = h, h+2, ...  Lane (rg, sub) copies
-    // the 16-byte chunk sub of every 128-byte segment of the rows rg, rg+4, ...
-    // so that 8 consecutive lanes read one segment; the feature indices of its
-    // rows sit in registers.
-    const int half = w, ht = lane;
+    // warps (half, part) fill stage half with the items i = half, half+2, ...;
+    // each of the two warps of a stage copies every other group of four rows.
+    // Lane (rg, sub) copies the 16-byte chunk sub of every 128-byte segment of
+    // its rows, so that 8 consecutive lanes read one segment; the feature
+    // indices of its rows sit in registers.
+    constexpr int P = kStepProd / 2;
+    constexpr int kRows = kRowsPerThr / P;
+    const int half = w & 1, part = w >> 1, ht = lane;
     const int sub = ht & 7, rg = ht >> 3;
     const uint32_t xg = XG(half), wg = WG(half);
     int i = half;
     for (; i < n_items; i += 2) {
       const int64_t g = gb + i;
       // the index loads are in flight while this half waits for its stage
-      int idx_cur[kRowsPerThr];
+      int idx_cur[kRows];
 #pragma unroll
-      for (int m = 0; m < kRowsPerThr; ++m) idx_cur[m] = a.idx[g * kK + rg + 4 * m];
+      for (int m = 0; m < kRows; ++m) idx_cur[m] = a.idx[g * kK + rg + 4 * (m * P + part)];
       if (!wait_or_abort(&empty[half], ((i >> 1) & 1) ^ 1, abort_flag)) break;
       const int nbb = Bp / 64;
 #pragma unroll
-      for (int m = 0; m < kRowsPerThr; ++m) {
-        const int sl = rg + 4 * m;
+      for (int m = 0; m < kRows; ++m) {
+        const int sl = rg + 4 * (m * P + part);
         const __nv_bfloat16* src = Xt + (int64_t)idx_cur[m] * Bp + sub * 8;
         const uint32_t dst = xg + sw128((uint32_t)(sl * 128 + sub * 16));  // swizzle is the same in every block
 #pragma unroll
         for (int bb = 0; bb < 4; ++bb)
           if (bb < nbb) cp_async16(dst + (uint32_t)(bb * kK * 128), src + bb * 64, 16);
       }
-      // weight block of the group (contiguous G x k)
+      // weight block of the group (contiguous G x k), chunks split between the warps
       const __nv_bfloat16* wsrc = W + g * (int64_t)kG * kK;
       constexpr int cpr = kK / 8;
 #pragma unroll 4
-      for (int c0 = 0; c0 < kG * cpr; c0 += 32) {
+      for (int c0 = 32 * part; c0 < kG * cpr; c0 += 32 * P) {
         const int c = c0 + ht;
         const int j = c / cpr, cc = c % cpr;
         cp_async16(wg + sw128((uint32_t)((cc >> 3) * kG * 128 + j * 128 + (cc & 7) * 16)),
@@ -218,7 +227,7 @@ __global__ void __launch_bounds__(kStepThreads, 1)
       publish_all(&full[half]);
     }
     cp_async_wait_all();
-  } else if (w == 2) {
+  } else if (w == kStepMma) {
     // ------------------------------------------------------------ MMA issuer
     const uint32_t idesc_f = make_idesc(1, 1, 0, 128, kG);
     const uint32_t idesc_w = make_idesc(1, 0, 1, 128, kG);
@@ -263,7 +272,7 @@ __global__ void __launch_bounds__(kStepThreads, 1)
   } else {
     // ------------------------------------------------------------- epilogue
     // warp (q, hh): TMEM lane quarter q, label columns [hh*CH, hh*CH + CH)
-    const int ew = w - 3, q = w & 3, hh = ew >> 2;
+    const int ew = w - kStepMma - 1, q = w & 3, hh = ew >> 2;
     const int r = q * 32 + lane;  // row inside a 128-row tile (and dW slot)
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     const float scale = a.grad_scale;
@@ -294,6 +303,7 @@ __global__ void __launch_bounds__(kStepThreads, 1)
         if (t >= n_bt) break;
         const int b = t * 128 + r;
         const bool live = b < sh.B;
+        const float sl = live ? scale : 0.f, hs = 0.5f * sl;  // rows beyond B get dY = 0
         uint32_t ym = 0;
 #pragma unroll
         for (int e = 0; e < kMaxPosReg; ++e) {
@@ -311,16 +321,28 @@ __global__ void __launch_bounds__(kStepThreads, 1)
           if constexpr (NC == 8) tmem_ld8(F(s) + lane_off + (uint32_t)(t * kG + hh * CH + c), z);
           else tmem_ld16(F(s) + lane_off + (uint32_t)(t * kG + hh * CH + c), z);
           tmem_wait_ld();
-          float dyv[16], lin = 0.f, prod = 1.f;
+          // y = 0 everywhere first (positives are rare), then the few positive
+          // columns are corrected: dY -= scale, loss -= z.
+          float dyv[16], relu = 0.f, prod = 1.f;
 #pragma unroll
           for (int e = 0; e < NC; ++e) {
-            const float y = ((ym >> (c + e)) & 1u) ? 1.f : 0.f;
-            const float th = tanh_approx(0.5f * z[e]);
-            dyv[e] = live ? scale * (fmaf(0.5f, th, 0.5f) - y) : 0.f;
-            lin += fmaxf(z[e], 0.f) - z[e] * y;
-            prod *= fmaf(0.5f, fabsf(th), 0.5f);
+            const float th = tanh_approx(0.5f * z[e]);   // sigma(z) = (1 + th) / 2
+            dyv[e] = fmaf(hs, th, hs);                   // scale * sigma(z)
+            relu += fmaxf(z[e], 0.f);
+            prod *= fmaf(0.5f, fabsf(th), 0.5f);         // sigma(|z|)
           }
-          if (live) loss_acc += lin - __logf(prod);
+          float zy = 0.f;
+          const uint32_t yc = (ym >> c) & ((1u << NC) - 1u);
+          if (yc) {
+#pragma unroll
+            for (int e = 0; e < NC; ++e)
+              if ((yc >> e) & 1u) {
+                dyv[e] -= sl;
+                zy += z[e];
+              }
+          }
+          // softplus(z) - z y = max(z, 0) - log sigma(|z|) - z y
+          if (live) loss_acc += relu - zy - __logf(prod);
 #pragma unroll
           for (int hq = 0; hq < NC / 8; ++hq) {
             const uint4 v = make_uint4(pack_bf16x2(dyv[8 * hq], dyv[8 * hq + 1]),
@@ -371,7 +393,7 @@ __global__ void __launch_bounds__(kStepThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (w == 2) {
+  if (w == kStepMma) {
     tc_fence_after();
     tmem_dealloc(tmem, ncols);
   }
@@ -379,20 +401,26 @@ __global__ void __launch_bounds__(kStepThreads, 1)
 
 // ============================================================== k_dx2
 constexpr int kDxThreads = 672;  // 4 producer warps, MMA warp, 16 scatter warps
-constexpr int kZBufs = 4;        // Z buffers in TMEM (kK columns each)
+constexpr int kZBufs = 4;        // Z^T buffers in TMEM (128 columns each)
 
 // One CTA owns a band [f0, f1) of input features for a 128-row batch tile and a
-// chunk of groups.  For each group that has slots in the band:
-//   producers (warps 0-3): dY tile (128 x G) and the weight columns of the band's
-//     slots into a stage of the shared-memory ring (cp.async, completion tracked
-//     by the stage's mbarrier); warp 0 writes the slot -> accumulator-column map;
-//   MMA (warp 4): Z = dY_g W_g[:, slots] (128 x N, fp32) into one of four TMEM
-//     buffers;
-//   scatter (warps 5-20): each warp owns 32 batch rows x a quarter of the band and
-//     adds its Z columns into the fp32 band accumulator in shared memory.
-// Feature ownership is fixed per warp, so warps on different groups never touch
-// the same accumulator element; the slot order within a group is the index
-// order, so each accumulator element sums its terms in group order.
+// chunk of groups.  For each group with slots [lo, hi) in the band:
+//   producers (warps 0-3): the dY tile (128 x G) and the weight columns of slots
+//     [s0, hi), s0 = lo rounded down to 8, into a stage of the shared-memory ring
+//     (cp.async; each thread's copies arrive on the stage's mbarrier when they
+//     land); warp 0 writes each slot's feature into a 16-entry metadata ring;
+//   MMA (warp 4): Z^T = W_g[:, s0 + m]^T . dY_g^T (M = 128 slot rows, N = 128
+//     batch columns, K = G) into one of four TMEM buffers: TMEM lane m holds slot
+//     s0 + m, column b holds batch row b;
+//   scatter (warps 5-20): team h (four warps, one per TMEM lane quarter) owns
+//     batch columns [32h, 32h+32); each thread takes one slot and adds its 32 Z^T
+//     values into the feature's row of the fp32 band accumulator with 16-byte
+//     shared-memory accesses.  Slots of one group hold distinct features, and a
+//     team finishes a group before it starts the next, so every accumulator
+//     element receives its group terms one at a time, in ascending group order.
+// Accumulator: [band][128] fp32, 512-byte rows; the 16-byte chunk c of row f is
+// stored at chunk c ^ (f & 7), so the lanes of a warp (different features) spread
+// over the banks.
 template <int kG, int kK>
 __global__ void __launch_bounds__(kDxThreads, 1)
     k_dx2(DxArgs a, const __nv_bfloat16* __restrict__ dY, const __nv_bfloat16* __restrict__ W) {
@@ -414,7 +442,7 @@ __global__ void __launch_bounds__(kDxThreads, 1)
   const DxLayout Lo = dx_layout(a.band, kK, kG, NS);
   const uint32_t base = align1024(smem_u32(smem));
   uint8_t* gbase = smem + (base - smem_u32(smem));
-  float* acc = reinterpret_cast<float*>(gbase + Lo.acc);  // [band][128] fp32
+  uint8_t* acc = gbase + Lo.acc;  // [band][128] fp32, chunk-swizzled rows
   auto meta = [&](int ms) -> int32_t* { return reinterpret_cast<int32_t*>(gbase + Lo.meta + ms * Lo.meta_stride); };
   auto DYS = [&](int ds) -> uint32_t { return base + Lo.dy + ds * Lo.dy_stride; };
   auto WS = [&](int ds) -> uint32_t { return base + Lo.w + ds * Lo.w_stride; };
@@ -423,9 +451,10 @@ __global__ void __launch_bounds__(kDxThreads, 1)
   uint64_t* empty = full + kMaxDxStages;          // [NS] stage consumed by the MMA
   uint64_t* meta_full = empty + kMaxDxStages;     // [16] metadata written (count: warp 0)
   uint64_t* meta_empty = meta_full + kMetaSlots;  // [16] metadata consumed by the scatter
-  uint64_t* z_full = meta_empty + kMetaSlots;     // [4] Z in TMEM
-  uint64_t* z_empty = z_full + kZBufs;            // [4] Z read out
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(z_empty + kZBufs);
+  uint64_t* z_full = meta_empty + kMetaSlots;     // [4] Z^T in TMEM
+  uint64_t* z_empty = z_full + kZBufs;            // [4] Z^T read out
+  uint64_t* team = z_empty + kZBufs;              // [4] a scatter team finished a group
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(team + 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
 
   const int w = warp_id(), lane = lane_id();
@@ -442,10 +471,11 @@ __global__ void __launch_bounds__(kDxThreads, 1)
       mbar_init(&z_full[s], 1);
       mbar_init(&z_empty[s], 16);
     }
+    for (int s = 0; s < 4; ++s) mbar_init(&team[s], 4);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  constexpr uint32_t kTmemCols = kZBufs * kK;
+  constexpr uint32_t kTmemCols = kZBufs * 128;
   if (w == 4) {
     tmem_alloc(tslot, kTmemCols);
     tmem_relinquish();
@@ -454,16 +484,13 @@ __global__ void __launch_bounds__(kDxThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tslot;
-  auto Z = [&](int s) -> uint32_t { return tmem + (uint32_t)(s * kK); };
-  // feature quarters of the band: [fq(j), fq(j+1)) belongs to scatter warps with p = j
-  auto fq = [&](int j) -> int { return min(f1, f0 + (a.band * j) / 4); };
+  auto Z = [&](int s) -> uint32_t { return tmem + (uint32_t)(s * 128); };
 
   if (w < 4) {
     // ------------------------------------------------- cp.async producers
     // Each producer warp reads the group's index row itself (two rows ahead) and
-    // derives the band's slot split points (idx is sorted); warp 0 also writes
-    // the metadata.  Each thread's copies of a stage arrive on the stage's full
-    // barrier when they land, so up to NS stages are in flight.
+    // finds the band's slot range [lo, hi) by ballots (idx is sorted); warp 0
+    // also writes the metadata.
     const int tid = threadIdx.x;
     int va[kPf], vb[kPf];  // index rows of groups g (even offset) and g + 1 (odd offset)
 #pragma unroll
@@ -476,13 +503,12 @@ __global__ void __launch_bounds__(kDxThreads, 1)
     // One group: v holds its index row on entry and the row of g + 2 on exit (the
     // load is only consumed two groups later, so its latency stays hidden).
     auto produce = [&](int64_t g, int (&v)[kPf]) -> bool {
-      int cnt[5] = {0, 0, 0, 0, 0};
+      int lo = 0, hi = 0;
 #pragma unroll
       for (int j = 0; j < kPf; ++j) {
-#pragma unroll
-        for (int e = 0; e < 5; ++e) cnt[e] += __popc(__ballot_sync(0xffffffffu, v[j] < fq(e)));
+        lo += __popc(__ballot_sync(0xffffffffu, v[j] < f0));
+        hi += __popc(__ballot_sync(0xffffffffu, v[j] < f1));
       }
-      const int lo = cnt[0], hi = cnt[4];
       const int ms = i % kMetaSlots;
       if (hi > lo && w == 0) {
         if (!wait_or_abort(&meta_empty[ms], ((i / kMetaSlots) & 1) ^ 1, abort_flag)) return false;
@@ -490,7 +516,7 @@ __global__ void __launch_bounds__(kDxThreads, 1)
 #pragma unroll
         for (int j = 0; j < kPf; ++j) {
           const int sl = lane + 32 * j;
-          if (sl >= lo && sl < hi) m[kMetaHdr + sl - lo] = (v[j] - f0) * 128;  // accumulator row offset
+          if (sl >= lo && sl < hi) m[kMetaHdr + sl - lo] = v[j] - f0;  // accumulator row
         }
       }
       if (g + 2 < g1) {
@@ -498,14 +524,16 @@ __global__ void __launch_bounds__(kDxThreads, 1)
         for (int j = 0; j < kPf; ++j) v[j] = a.idx[(g + 2) * kK + lane + 32 * j];  // prefetch
       }
       if (hi == lo) return true;  // no feature of this band in the group (uniform)
-      const int s0 = lo & ~63;
-      const int nblk = (hi - s0 + 63) / 64;  // 64-slot blocks of weight columns
+      // slot rows of Z^T start at s0 = lo rounded down to 8; hi - s0 <= k <= 128
+      const int s0 = lo & ~7;
+      const int nch = (hi - s0 + 7) >> 3;  // 8-slot chunks of weight columns
       if (w == 0) {
         int32_t* m = meta(ms);
-        if (lane < 5) m[lane] = lane == 0 ? cnt[0] : lane == 1 ? cnt[1] : lane == 2 ? cnt[2] : lane == 3 ? cnt[3] : cnt[4];
         if (lane == 0) {
+          m[0] = lo;
           m[5] = s0;
-          m[6] = nblk * 64;
+          m[6] = 1;  // a group (0: end of the chunk)
+          m[7] = hi;
         }
         __syncwarp();
         mbar_arrive(&meta_full[ms]);
@@ -524,17 +552,17 @@ __global__ void __launch_bounds__(kDxThreads, 1)
         cp_async16(dys + swz_rows((uint32_t)(b * RB + cc * 16), RB),
                    in ? dyg + (int64_t)row * a.dy_rstride + cc * 8 : dY, in ? 16u : 0u);
       }
-      // weight columns [s0, s0 + 64*nblk) of the group's G x k block
+      // weight chunks [s0, s0 + 8 nch) of the group's G x k block: row j (label),
+      // chunk cr -> M block cr / 8 of the swizzled MN-major tile
       const uint32_t ws = WS(ds);
       const __nv_bfloat16* wsrc = W + g * (int64_t)kG * kK + s0;
-      for (int blk = 0; blk < nblk; ++blk) {
 #pragma unroll
-        for (int r = 0; r < kG / 16; ++r) {
-          const int qq = tid + 128 * r;
-          const int j = qq >> 3, cc = qq & 7;
-          cp_async16(ws + (uint32_t)(blk * kG * 128) + sw128((uint32_t)(j * 128 + cc * 16)),
-                     wsrc + (int64_t)j * kK + blk * 64 + cc * 8, 16);
-        }
+      for (int q0 = 0; q0 < kG * 16; q0 += 128) {
+        const int qq = q0 + tid;
+        const int j = qq >> 4, cr = qq & 15;
+        if (cr < nch)
+          cp_async16(ws + (uint32_t)((cr >> 3) * kG * 128) + sw128((uint32_t)(j * 128 + (cr & 7) * 16)),
+                     wsrc + (int64_t)j * kK + cr * 8, 16);
       }
       cp_async_arrive_on(&full[ds]);  // the stage publishes itself when its copies land
       ++i;
@@ -552,7 +580,7 @@ __global__ void __launch_bounds__(kDxThreads, 1)
     }
     cp_async_wait_all();
     if (!stopped) {
-      // end marker: metadata N = 0 and a data stage without copies
+      // end marker: metadata 0 and a data stage without copies
       const int ms = i % kMetaSlots;
       if (wait_or_abort(&empty[ds], dph ^ 1, abort_flag)) {
         if (w == 0 && wait_or_abort(&meta_empty[ms], ((i / kMetaSlots) & 1) ^ 1, abort_flag)) {
@@ -565,21 +593,20 @@ __global__ void __launch_bounds__(kDxThreads, 1)
     }
   } else if (w == 4) {
     // ------------------------------------------------------------- MMA
+    const uint32_t idesc = make_idesc(1, 1, 0, 128, 128);
     int ds = 0, dph = 0;
     for (int i = 0;; ++i) {
       const int ms = i % kMetaSlots, zs = i % kZBufs;
       if (!wait_or_abort(&full[ds], dph, abort_flag)) break;
       if (!wait_or_abort(&meta_full[ms], (i / kMetaSlots) & 1, abort_flag)) break;
       fence_proxy_async_smem();  // landed cp.async data is read by the tensor core
-      const int N = *reinterpret_cast<volatile int32_t*>(&meta(ms)[6]);
-      if (N == 0) break;
+      if (*reinterpret_cast<volatile int32_t*>(&meta(ms)[6]) == 0) break;
       if (!wait_or_abort(&z_empty[zs], ((i / kZBufs) & 1) ^ 1, abort_flag)) break;
       tc_fence_after();
       if (lane == 0) {
-        const uint32_t idesc = make_idesc(1, 0, 1, 128, (uint32_t)N);
         for (int kk = 0; kk < kG / 16; ++kk) {
-          const uint64_t ad = make_sdesc(DYS(ds) + (uint32_t)(kk * 32), 16, 8 * RB, layout_for_rows(RB));
-          const uint64_t bd = make_sdesc(WS(ds) + (uint32_t)(kk * 16 * 128), (uint32_t)kG * 128, 1024, kLayoutSw128);
+          const uint64_t ad = make_sdesc(WS(ds) + (uint32_t)(kk * 16 * 128), (uint32_t)kG * 128, 1024, kLayoutSw128);
+          const uint64_t bd = make_sdesc(DYS(ds) + (uint32_t)(kk * 32), 16, 8 * RB, layout_for_rows(RB));
           mma_ss<false>(Z(zs), ad, bd, idesc, kk > 0 ? 1u : 0u);
         }
         mma_commit(&z_full[zs]);
@@ -593,65 +620,63 @@ __global__ void __launch_bounds__(kDxThreads, 1)
     }
   } else {
     // ---------------------------------------------------------- scatter
-    const int q = w & 3, p = (w - 5) >> 2;  // batch quarter, feature quarter
-    const int b = q * 32 + lane;
+    const int q = w & 3, hb = (w - 5) >> 2;  // TMEM lane quarter, batch quarter (team)
+    const int st = threadIdx.x - 160;        // 0..511 over the scatter warps
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-    float* accb = acc + b;
-    for (int f = fq(p); f < fq(p + 1); ++f) accb[(f - f0) * 128] = 0.f;
+    const int nf = f1 - f0;
+    for (int e = st; e < nf * 32; e += 512) reinterpret_cast<float4*>(acc)[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+    named_bar(1, 512);
     for (int i = 0;; ++i) {
       const int ms = i % kMetaSlots, zs = i % kZBufs;
       if (!wait_or_abort(&meta_full[ms], (i / kMetaSlots) & 1, abort_flag)) break;
       const int32_t* m = meta(ms);
-      const int N = *reinterpret_cast<const volatile int32_t*>(&m[6]);
-      if (N == 0) break;
-      const int lo = m[0], beg = m[p], end = m[p + 1], s0 = m[5];
-      const int32_t* mo = m + kMetaHdr - lo;  // accumulator row offset of slot sl: mo[sl]
-      // Every warp waits for Z before it releases the buffer, also without slots
-      // in this group: a release may only count toward this group's phase.
-      if (!wait_or_abort(&z_full[zs], (i / kZBufs) & 1, abort_flag)) break;
-      tc_fence_after();
-      const uint32_t zcol = Z(zs) + lane_off - (uint32_t)s0;  // TMEM address of slot sl: zcol + sl
-      auto release_z = [&]() {
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&z_empty[zs]);
-      };
-      int sl = beg;
-      if (sl >= end) release_z();
-      for (; sl + 8 <= end; sl += 8) {  // full batches of 8 slots
-        float v[8];
-        int off[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) v[e] = tmem_ld1(zcol + (uint32_t)(sl + e));
-#pragma unroll
-        for (int e = 0; e < 8; ++e) off[e] = mo[sl + e];
-        tmem_wait_ld();
-        if (sl + 8 == end) release_z();
-#pragma unroll
-        for (int e = 0; e < 8; ++e) accb[off[e]] += v[e];
-      }
-      if (sl < end) {  // the last 1..7 slots (warp-uniform branches)
-        const int n = end - sl;
-        float v[7];
-        int off[7];
-#pragma unroll
-        for (int e = 0; e < 7; ++e)
-          if (e < n) v[e] = tmem_ld1(zcol + (uint32_t)(sl + e));
-#pragma unroll
-        for (int e = 0; e < 7; ++e)
-          if (e < n) off[e] = mo[sl + e];
-        tmem_wait_ld();
-        release_z();
-#pragma unroll
-        for (int e = 0; e < 7; ++e)
-          if (e < n) accb[off[e]] += v[e];
-      }
+      if (*reinterpret_cast<const volatile int32_t*>(&m[6]) == 0) break;
+      const int lo = m[0], s0 = m[5], hi = m[7];
+      const int sl = s0 + q * 32 + lane;  // this thread's slot
+      const bool act = sl >= lo && sl < hi;
+      const int f = act ? m[kMetaHdr + sl - lo] : 0;
       __syncwarp();
       if (lane == 0) mbar_arrive(&meta_empty[ms]);
+      if (!wait_or_abort(&z_full[zs], (i / kZBufs) & 1, abort_flag)) break;
+      tc_fence_after();
+      const bool any = __any_sync(0xffffffffu, act);
+      float v[32];
+      if (any) {
+        float* v0 = v;
+        float* v1 = v + 16;
+        tmem_ld16(Z(zs) + lane_off + (uint32_t)(32 * hb), *reinterpret_cast<float(*)[16]>(v0));
+        tmem_ld16(Z(zs) + lane_off + (uint32_t)(32 * hb + 16), *reinterpret_cast<float(*)[16]>(v1));
+        tmem_wait_ld();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&z_empty[zs]);
+      if (act) {
+        uint8_t* row = acc + (uint32_t)f * 512u;
+#pragma unroll
+        for (int cq = 0; cq < 8; ++cq) {
+          float4* p = reinterpret_cast<float4*>(row + (uint32_t)(((8 * hb + cq) ^ (f & 7)) * 16));
+          float4 o = *p;
+          o.x += v[4 * cq];
+          o.y += v[4 * cq + 1];
+          o.z += v[4 * cq + 2];
+          o.w += v[4 * cq + 3];
+          *p = o;
+        }
+      }
+      // the team finishes this group before any of its warps starts the next
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&team[hb]);
+      if (!wait_or_abort(&team[hb], i & 1, abort_flag)) break;
     }
-    // this warp's features x batch rows -> chunk partial
-    for (int f = fq(p); f < fq(p + 1); ++f)
-      a.dX_part[((int64_t)c * sh.d + f) * sh.Bp + t * 128 + b] = accb[(f - f0) * 128];
+    named_bar(1, 512);
+    // band accumulator -> chunk partial (un-swizzled, coalesced over batch rows)
+    for (int e = st; e < nf * 128; e += 512) {
+      const int fr = e >> 7, b = e & 127;
+      const float val = *reinterpret_cast<const float*>(acc + (uint32_t)fr * 512u +
+                                                        (uint32_t)((((b >> 2) ^ (fr & 7)) * 16) + (b & 3) * 4));
+      a.dX_part[((int64_t)c * sh.d + f0 + fr) * sh.Bp + t * 128 + b] = val;
+    }
   }
   tc_fence_before();
   __syncthreads();
