@@ -43,6 +43,8 @@ struct DxArgs {
   int band, n_bands, n_chunks, ns;  // ns: stages of the shared-memory ring
   // element (b, g*G + j) of dY is at dY[g*dy_gstride + b*dy_rstride + j]
   int64_t dy_gstride, dy_rstride;
+  // dY tile of group g, batch tile t in the dY tensor map: x = g*dy_xg, y = g*dy_yg + 128 t
+  int dy_xg, dy_yg;
 };
 
 constexpr int kMetaSlots = 16;  // metadata ring of the dX pass (twice the deepest data ring)
@@ -81,7 +83,7 @@ __host__ __device__ inline DxLayout dx_layout(int band, int k, int G, int ns) {
   // when k = 128 (hi - s0 <= k); with k = 64 the second block the MMA reads is the
   // next region of shared memory and feeds only TMEM lanes no thread reads.
   L.w_stride = (uint32_t)((k / 64) * G * 128);
-  L.meta_stride = (uint32_t)(kMetaHdr + k) * 4;
+  L.meta_stride = 0;
   uint32_t off = 0;
   L.dy = off;
   off += ns * L.dy_stride;
@@ -351,7 +353,7 @@ __global__ void __launch_bounds__(kStepThreads, 1)
                                        pack_bf16x2(dyv[8 * hq + 6], dyv[8 * hq + 7]));
             const int col = hh * CH + c + 8 * hq;
             *reinterpret_cast<uint4*>(dyrow + swz_rows((uint32_t)(b * RB + col * 2), RB)) = v;
-            if (live) *reinterpret_cast<uint4*>(dyg + (int64_t)b * kG + col) = v;
+            *reinterpret_cast<uint4*>(dyg + (int64_t)b * kG + col) = v;  // rows past B: zeros
           }
         }
       }
@@ -400,33 +402,35 @@ __global__ void __launch_bounds__(kStepThreads, 1)
 }
 
 // ============================================================== k_dx2
-constexpr int kDxThreads = 672;  // 4 producer warps, MMA warp, 16 scatter warps
+constexpr int kDxThreads = 576;  // producer warp, MMA warp, 16 scatter warps
 constexpr int kZBufs = 4;        // Z^T buffers in TMEM (128 columns each)
 
 // One CTA owns a band [f0, f1) of input features for a 128-row batch tile and a
-// chunk of groups.  For each group with slots [lo, hi) in the band:
-//   producers (warps 0-3): the dY tile (128 x G) and the weight columns of slots
-//     [s0, hi), s0 = lo rounded down to 8, into a stage of the shared-memory ring
-//     (cp.async; each thread's copies arrive on the stage's mbarrier when they
-//     land); warp 0 writes each slot's feature into a 16-entry metadata ring;
-//   MMA (warp 4): Z^T = W_g[:, s0 + m]^T . dY_g^T (M = 128 slot rows, N = 128
-//     batch columns, K = G) into one of four TMEM buffers: TMEM lane m holds slot
-//     s0 + m, column b holds batch row b;
-//   scatter (warps 5-20): team h (four warps, one per TMEM lane quarter) owns
-//     batch columns [32h, 32h+32); each thread takes one slot and adds its 32 Z^T
-//     values into the feature's row of the fp32 band accumulator with 16-byte
-//     shared-memory accesses.  Slots of one group hold distinct features, and a
-//     team finishes a group before it starts the next, so every accumulator
-//     element receives its group terms one at a time, in ascending group order.
+// chunk of groups.  For every group g of the chunk:
+//   producer (warp 0, one thread): the dY tile (128 x G) and the whole G x k
+//     weight block into a stage of the shared-memory ring with TMA (2D tiles,
+//     hardware swizzle, zero fill past the tensor's edges);
+//   MMA (warp 1): Z^T = W_g^T . dY_g^T (M = 128 slot rows, N = 128 batch columns,
+//     K = G) into one of four TMEM buffers: TMEM lane s holds slot s of the group;
+//   scatter (warps 2-17): team h (four warps, one per TMEM lane quarter) owns
+//     batch columns [32h, 32h+32).  The thread of slot s reads the slot's feature
+//     from the index array itself (a few groups ahead) and, when it falls in the
+//     band, adds its 32 Z^T values into the feature's row of the fp32 band
+//     accumulator with 16-byte shared-memory accesses.  Slots of one group hold
+//     distinct features, and a team finishes a group (named barrier) before it
+//     starts the next, so every accumulator element receives its group terms one
+//     at a time, in ascending group order.
+// Every warp runs the same number of iterations (one per group of the chunk), so
+// the named barriers always match; a wait that runs out raises the abort flag and
+// the remaining iterations skip their work.
 // Accumulator: [band][128] fp32, 512-byte rows; the 16-byte chunk c of row f is
 // stored at chunk c ^ (f & 7), so the lanes of a warp (different features) spread
 // over the banks.
 template <int kG, int kK>
 __global__ void __launch_bounds__(kDxThreads, 1)
-    k_dx2(DxArgs a, const __nv_bfloat16* __restrict__ dY, const __nv_bfloat16* __restrict__ W) {
+    k_dx2(DxArgs a, const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__ CUtensorMap tm_w) {
   extern __shared__ __align__(1024) uint8_t smem[];
   constexpr int RB = kG * 2;
-  constexpr int kPf = kK / 32;  // index registers per lane for one group row
   const int NS = a.ns;
   const TailShape sh = a.sh;
   const int n_bt = sh.Bp / 128;
@@ -438,45 +442,37 @@ __global__ void __launch_bounds__(kDxThreads, 1)
   const int f1 = min(sh.d, f0 + a.band);
   const int64_t g0 = (int64_t)c * sh.n_groups / a.n_chunks;
   const int64_t g1 = (int64_t)(c + 1) * sh.n_groups / a.n_chunks;
+  const int n = (int)(g1 - g0);
 
   const DxLayout Lo = dx_layout(a.band, kK, kG, NS);
   const uint32_t base = align1024(smem_u32(smem));
   uint8_t* gbase = smem + (base - smem_u32(smem));
   uint8_t* acc = gbase + Lo.acc;  // [band][128] fp32, chunk-swizzled rows
-  auto meta = [&](int ms) -> int32_t* { return reinterpret_cast<int32_t*>(gbase + Lo.meta + ms * Lo.meta_stride); };
   auto DYS = [&](int ds) -> uint32_t { return base + Lo.dy + ds * Lo.dy_stride; };
   auto WS = [&](int ds) -> uint32_t { return base + Lo.w + ds * Lo.w_stride; };
   uint64_t* bars = reinterpret_cast<uint64_t*>(gbase + Lo.bars);
-  uint64_t* full = bars;                          // [NS] stage landed (count: 128 producer threads)
-  uint64_t* empty = full + kMaxDxStages;          // [NS] stage consumed by the MMA
-  uint64_t* meta_full = empty + kMaxDxStages;     // [16] metadata written (count: warp 0)
-  uint64_t* meta_empty = meta_full + kMetaSlots;  // [16] metadata consumed by the scatter
-  uint64_t* z_full = meta_empty + kMetaSlots;     // [4] Z^T in TMEM
-  uint64_t* z_empty = z_full + kZBufs;            // [4] Z^T read out
-  uint64_t* team = z_empty + kZBufs;              // [4] a scatter team finished a group
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(team + 4);
+  uint64_t* full = bars;                  // [NS] stage landed (count: 1 + transaction bytes)
+  uint64_t* empty = full + kMaxDxStages;  // [NS] stage consumed by the MMA
+  uint64_t* z_full = empty + kMaxDxStages;  // [4] Z^T in TMEM
+  uint64_t* z_empty = z_full + kZBufs;      // [4] Z^T read out
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(z_empty + kZBufs);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
 
   const int w = warp_id(), lane = lane_id();
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
-      mbar_init(&full[s], 128);
+      mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
-    }
-    for (int s = 0; s < kMetaSlots; ++s) {
-      mbar_init(&meta_full[s], 32);
-      mbar_init(&meta_empty[s], 16);
     }
     for (int s = 0; s < kZBufs; ++s) {
       mbar_init(&z_full[s], 1);
       mbar_init(&z_empty[s], 16);
     }
-    for (int s = 0; s < 4; ++s) mbar_init(&team[s], 4);
     *abort_flag = 0;
     fence_mbar_init();
   }
   constexpr uint32_t kTmemCols = kZBufs * 128;
-  if (w == 4) {
+  if (w == 1) {
     tmem_alloc(tslot, kTmemCols);
     tmem_relinquish();
   }
@@ -486,122 +482,37 @@ __global__ void __launch_bounds__(kDxThreads, 1)
   const uint32_t tmem = *tslot;
   auto Z = [&](int s) -> uint32_t { return tmem + (uint32_t)(s * 128); };
 
-  if (w < 4) {
-    // ------------------------------------------------- cp.async producers
-    // Each producer warp reads the group's index row itself (two rows ahead) and
-    // finds the band's slot range [lo, hi) by ballots (idx is sorted); warp 0
-    // also writes the metadata.
-    const int tid = threadIdx.x;
-    int va[kPf], vb[kPf];  // index rows of groups g (even offset) and g + 1 (odd offset)
+  if (w == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      constexpr uint32_t kBytes = 128 * kG * 2 + (kK / 64) * 64 * kG * 2;
+      int ds = 0, dph = 0, issued = 0;
+      for (int i = 0; i < n; ++i) {
+        const int64_t g = g0 + i;
+        if (!wait_or_abort(&empty[ds], dph ^ 1, abort_flag)) break;
+        ++issued;
+        mbar_arrive_expect_tx(&full[ds], kBytes);
+        tma_load_2d(DYS(ds), &tm_dy, (int)(g * a.dy_xg), (int)(g * a.dy_yg) + 128 * t, &full[ds]);
 #pragma unroll
-    for (int j = 0; j < kPf; ++j) {
-      va[j] = g0 < g1 ? a.idx[g0 * kK + lane + 32 * j] : 0;
-      vb[j] = g0 + 1 < g1 ? a.idx[(g0 + 1) * kK + lane + 32 * j] : 0;
-    }
-    int i = 0, ds = 0, dph = 0;
-    bool stopped = false;
-    // One group: v holds its index row on entry and the row of g + 2 on exit (the
-    // load is only consumed two groups later, so its latency stays hidden).
-    auto produce = [&](int64_t g, int (&v)[kPf]) -> bool {
-      int lo = 0, hi = 0;
-#pragma unroll
-      for (int j = 0; j < kPf; ++j) {
-        lo += __popc(__ballot_sync(0xffffffffu, v[j] < f0));
-        hi += __popc(__ballot_sync(0xffffffffu, v[j] < f1));
-      }
-      const int ms = i % kMetaSlots;
-      if (hi > lo && w == 0) {
-        if (!wait_or_abort(&meta_empty[ms], ((i / kMetaSlots) & 1) ^ 1, abort_flag)) return false;
-        int32_t* m = meta(ms);
-#pragma unroll
-        for (int j = 0; j < kPf; ++j) {
-          const int sl = lane + 32 * j;
-          if (sl >= lo && sl < hi) m[kMetaHdr + sl - lo] = v[j] - f0;  // accumulator row
+        for (int blk = 0; blk < kK / 64; ++blk)
+          tma_load_2d(WS(ds) + (uint32_t)(blk * kG * 128), &tm_w, 64 * blk, (int)(g * kG), &full[ds]);
+        if (++ds == NS) {
+          ds = 0;
+          dph ^= 1;
         }
       }
-      if (g + 2 < g1) {
-#pragma unroll
-        for (int j = 0; j < kPf; ++j) v[j] = a.idx[(g + 2) * kK + lane + 32 * j];  // prefetch
-      }
-      if (hi == lo) return true;  // no feature of this band in the group (uniform)
-      // slot rows of Z^T start at s0 = lo rounded down to 8; hi - s0 <= k <= 128
-      const int s0 = lo & ~7;
-      const int nch = (hi - s0 + 7) >> 3;  // 8-slot chunks of weight columns
-      if (w == 0) {
-        int32_t* m = meta(ms);
-        if (lane == 0) {
-          m[0] = lo;
-          m[5] = s0;
-          m[6] = 1;  // a group (0: end of the chunk)
-          m[7] = hi;
-        }
-        __syncwarp();
-        mbar_arrive(&meta_full[ms]);
-      }
-      if (!wait_or_abort(&empty[ds], dph ^ 1, abort_flag)) return false;
-      // dY tile: 128 rows of G labels (rows at or beyond B read as zero)
-      const uint32_t dys = DYS(ds);
-      constexpr int cpr = kG / 8;
-      const __nv_bfloat16* dyg = dY + g * a.dy_gstride;
-#pragma unroll
-      for (int q0 = 0; q0 < 128 * cpr; q0 += 128) {
-        const int qq = q0 + tid;
-        const int b = qq / cpr, cc = qq % cpr;
-        const int row = t * 128 + b;
-        const bool in = row < sh.B;
-        cp_async16(dys + swz_rows((uint32_t)(b * RB + cc * 16), RB),
-                   in ? dyg + (int64_t)row * a.dy_rstride + cc * 8 : dY, in ? 16u : 0u);
-      }
-      // weight chunks [s0, s0 + 8 nch) of the group's G x k block: row j (label),
-      // chunk cr -> M block cr / 8 of the swizzled MN-major tile
-      const uint32_t ws = WS(ds);
-      const __nv_bfloat16* wsrc = W + g * (int64_t)kG * kK + s0;
-#pragma unroll
-      for (int q0 = 0; q0 < kG * 16; q0 += 128) {
-        const int qq = q0 + tid;
-        const int j = qq >> 4, cr = qq & 15;
-        if (cr < nch)
-          cp_async16(ws + (uint32_t)((cr >> 3) * kG * 128) + sw128((uint32_t)(j * 128 + (cr & 7) * 16)),
-                     wsrc + (int64_t)j * kK + cr * 8, 16);
-      }
-      cp_async_arrive_on(&full[ds]);  // the stage publishes itself when its copies land
-      ++i;
-      if (++ds == NS) {
-        ds = 0;
-        dph ^= 1;
-      }
-      return true;
-    };
-    for (int64_t g = g0; g < g1; g += 2) {
-      if (!produce(g, va) || (g + 1 < g1 && !produce(g + 1, vb))) {
-        stopped = true;
-        break;
-      }
+      // no copy may still be landing when the CTA exits (an abort can leave the
+      // last stages unconsumed)
+      for (int j = issued > NS ? issued - NS : 0; j < issued; ++j) mbar_wait(&full[j % NS], (j / NS) & 1);
     }
-    cp_async_wait_all();
-    if (!stopped) {
-      // end marker: metadata 0 and a data stage without copies
-      const int ms = i % kMetaSlots;
-      if (wait_or_abort(&empty[ds], dph ^ 1, abort_flag)) {
-        if (w == 0 && wait_or_abort(&meta_empty[ms], ((i / kMetaSlots) & 1) ^ 1, abort_flag)) {
-          if (lane == 0) meta(ms)[6] = 0;
-          __syncwarp();
-          mbar_arrive(&meta_full[ms]);
-        }
-        mbar_arrive(&full[ds]);
-      }
-    }
-  } else if (w == 4) {
+  } else if (w == 1) {
     // ------------------------------------------------------------- MMA
     const uint32_t idesc = make_idesc(1, 1, 0, 128, 128);
     int ds = 0, dph = 0;
-    for (int i = 0;; ++i) {
-      const int ms = i % kMetaSlots, zs = i % kZBufs;
-      if (!wait_or_abort(&full[ds], dph, abort_flag)) break;
-      if (!wait_or_abort(&meta_full[ms], (i / kMetaSlots) & 1, abort_flag)) break;
-      fence_proxy_async_smem();  // landed cp.async data is read by the tensor core
-      if (*reinterpret_cast<volatile int32_t*>(&meta(ms)[6]) == 0) break;
-      if (!wait_or_abort(&z_empty[zs], ((i / kZBufs) & 1) ^ 1, abort_flag)) break;
+    for (int i = 0; i < n; ++i) {
+      const int zs = i % kZBufs;
+      if (!__all_sync(0xffffffffu, wait_or_abort(&full[ds], dph, abort_flag))) break;
+      if (!__all_sync(0xffffffffu, wait_or_abort(&z_empty[zs], ((i / kZBufs) & 1) ^ 1, abort_flag))) break;
       tc_fence_after();
       if (lane == 0) {
         for (int kk = 0; kk < kG / 16; ++kk) {
@@ -620,38 +531,46 @@ __global__ void __launch_bounds__(kDxThreads, 1)
     }
   } else {
     // ---------------------------------------------------------- scatter
-    const int q = w & 3, hb = (w - 5) >> 2;  // TMEM lane quarter, batch quarter (team)
-    const int st = threadIdx.x - 160;        // 0..511 over the scatter warps
+    const int q = w & 3, hb = (w - 2) >> 2;  // TMEM lane quarter, batch quarter (team)
+    const int st = threadIdx.x - 64;         // 0..511 over the scatter warps
+    const int s = q * 32 + lane;             // this thread's slot
+    const bool slot_ok = s < kK;
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     const int nf = f1 - f0;
     for (int e = st; e < nf * 32; e += 512) reinterpret_cast<float4*>(acc)[e] = make_float4(0.f, 0.f, 0.f, 0.f);
-    named_bar(1, 512);
-    for (int i = 0;; ++i) {
-      const int ms = i % kMetaSlots, zs = i % kZBufs;
-      if (!wait_or_abort(&meta_full[ms], (i / kMetaSlots) & 1, abort_flag)) break;
-      const int32_t* m = meta(ms);
-      if (*reinterpret_cast<const volatile int32_t*>(&m[6]) == 0) break;
-      const int lo = m[0], s0 = m[5], hi = m[7];
-      const int sl = s0 + q * 32 + lane;  // this thread's slot
-      const bool act = sl >= lo && sl < hi;
-      const int f = act ? m[kMetaHdr + sl - lo] : 0;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&meta_empty[ms]);
-      if (!wait_or_abort(&z_full[zs], (i / kZBufs) & 1, abort_flag)) break;
-      tc_fence_after();
-      const bool any = __any_sync(0xffffffffu, act);
+    named_bar(5, 512);
+    // the slot's feature, three groups ahead in registers
+    int fa = 0, fb = 0, fc = 0;
+    if (slot_ok) {
+      if (n > 0) fa = a.idx[g0 * kK + s];
+      if (n > 1) fb = a.idx[(g0 + 1) * kK + s];
+      if (n > 2) fc = a.idx[(g0 + 2) * kK + s];
+    }
+    for (int i = 0; i < n; ++i) {
+      const int zs = i % kZBufs;
+      const int f = fa - f0;
+      const bool act = slot_ok && f >= 0 && f < nf;
+      fa = fb;
+      fb = fc;
+      if (slot_ok && i + 3 < n) fc = a.idx[(g0 + i + 3) * kK + s];
       float v[32];
-      if (any) {
-        float* v0 = v;
-        float* v1 = v + 16;
-        tmem_ld16(Z(zs) + lane_off + (uint32_t)(32 * hb), *reinterpret_cast<float(*)[16]>(v0));
-        tmem_ld16(Z(zs) + lane_off + (uint32_t)(32 * hb + 16), *reinterpret_cast<float(*)[16]>(v1));
-        tmem_wait_ld();
+      const bool ok = __all_sync(0xffffffffu, wait_or_abort(&z_full[zs], (i / kZBufs) & 1, abort_flag));
+      if (ok) {
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, act)) {
+          float* v0 = v;
+          float* v1 = v + 16;
+          tmem_ld16(Z(zs) + lane_off + (uint32_t)(32 * hb), *reinterpret_cast<float(*)[16]>(v0));
+          tmem_ld16(Z(zs) + lane_off + (uint32_t)(32 * hb + 16), *reinterpret_cast<float(*)[16]>(v1));
+          tmem_wait_ld();
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&z_empty[zs]);
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&z_empty[zs]);
-      if (act) {
+      // the team finishes group i-1 before any of its warps adds group i
+      named_bar(1 + hb, 128);
+      if (ok && act) {
         uint8_t* row = acc + (uint32_t)f * 512u;
 #pragma unroll
         for (int cq = 0; cq < 8; ++cq) {
@@ -664,12 +583,8 @@ __global__ void __launch_bounds__(kDxThreads, 1)
           *p = o;
         }
       }
-      // the team finishes this group before any of its warps starts the next
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&team[hb]);
-      if (!wait_or_abort(&team[hb], i & 1, abort_flag)) break;
     }
-    named_bar(1, 512);
+    named_bar(5, 512);
     // band accumulator -> chunk partial (un-swizzled, coalesced over batch rows)
     for (int e = st; e < nf * 128; e += 512) {
       const int fr = e >> 7, b = e & 127;
@@ -680,7 +595,7 @@ __global__ void __launch_bounds__(kDxThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (w == 4) {
+  if (w == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
@@ -728,15 +643,69 @@ cudaError_t launch_step_t(const v2::StepArgs& a, int grid, const void* Xt, const
   return cudaGetLastError();
 }
 
+// cuTensorMapEncodeTiled from the driver, looked up once through the runtime.
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_tiled() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2D bf16 tensor map: `inner` contiguous elements per row, `outer` rows of
+// `row_bytes` bytes; box of box_inner x box_outer elements, read past the edges as
+// zeros.  The swizzle follows the box row width (32, 64 or 128 bytes).
+cudaError_t tmap_2d(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+                    uint32_t box_inner, uint32_t box_outer) {
+  EncodeTiledFn enc = encode_tiled();
+  if (!enc) return cudaErrorNotSupported;
+  const uint32_t rb = box_inner * 2;
+  const CUtensorMapSwizzle sw = rb == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                : rb == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                           : CU_TENSOR_MAP_SWIZZLE_32B;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+// dY of the dX pass, either the group-major buffer [n_groups, Bp, G] of the fused
+// step (dy_gstride = Bp*G, dy_rstride = G; rows past B hold zeros) or a caller's
+// row-major [B, L] (dy_gstride = G, dy_rstride = L; rows past B are outside the
+// tensor and read as zeros).
 template <int kG, int kK>
-cudaError_t launch_dx_t(const v2::DxArgs& a, const void* dY, const void* W, cudaStream_t st) {
+cudaError_t launch_dx_t(v2::DxArgs a, const void* dY, const void* W, cudaStream_t st) {
   const size_t smem = dx_smem(a.band, kK, kG, a.ns);
   auto kern = v2::k_dx2<kG, kK>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
+  CUtensorMap tm_dy, tm_w;
+  const bool group_major = a.dy_gstride != kG;  // row-major [B, L] has dy_gstride = G
+  if (group_major) {
+    e = tmap_2d(&tm_dy, dY, kG, (uint64_t)a.sh.n_groups * a.sh.Bp, (uint64_t)kG * 2, kG, 128);
+    a.dy_xg = 0;
+    a.dy_yg = a.sh.Bp;
+  } else {
+    e = tmap_2d(&tm_dy, dY, (uint64_t)a.sh.L, (uint64_t)a.sh.B, (uint64_t)a.dy_rstride * 2, kG, 128);
+    a.dy_xg = kG;
+    a.dy_yg = 0;
+  }
+  if (e == cudaSuccess) e = tmap_2d(&tm_w, W, kK, (uint64_t)a.sh.L, (uint64_t)kK * 2, 64, kG);
+  if (e != cudaSuccess) return e;
   const int grid = (a.sh.Bp / 128) * a.n_bands * a.n_chunks;
-  kern<<<grid, v2::kDxThreads, smem, st>>>(a, static_cast<const __nv_bfloat16*>(dY),
-                                           static_cast<const __nv_bfloat16*>(W));
+  kern<<<grid, v2::kDxThreads, smem, st>>>(a, tm_dy, tm_w);
   return cudaGetLastError();
 }
 
