@@ -78,6 +78,26 @@ def algorithmic(wl):
     return out
 
 
+# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) of the
+# dominant kernel from one ncu capture (summaries under profiles/), valid only for
+# the kernel source they were taken on: (config, kernel) -> (bytes, source digest).
+TRAFFIC = {
+    ("670k", "tail_dx"): (529.2e6, "f00a0980e567a9e1"),
+}
+KERNEL_SOURCE = os.path.join(ROOT, "structured_sparse_output_b200", "csrc", "tail_v2.cu")
+
+
+def traffic_of(config, kernel):
+    """The captured traffic, or None when the kernel source changed since the capture."""
+    import hashlib
+    got = TRAFFIC.get((config, kernel))
+    if got is None or not os.path.exists(KERNEL_SOURCE):
+        return None
+    with open(KERNEL_SOURCE, "rb") as fh:
+        digest = hashlib.sha256(fh.read()).hexdigest()[:16]
+    return got[0] if digest == got[1] else None
+
+
 def roofline_of(flops, nbytes, ms, peaks, sustained=True):
     tf = peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"]
     t_tensor = flops / (tf * 1e12)
@@ -410,7 +430,8 @@ def main():
     rf["kernel"] = dom
     rf["ms_per_launch"] = round(tot_ms / n_l, 4)
     rf["peak_src"] = f"{peaks['src']} ({'sustained' if rf['bound'] == 'tensor' else 'copy'})"
-    rf["traffic"] = None
+    rf["traffic"] = traffic_of(args.config, dom)
+    rf["traffic_src"] = "ncu capture, profiles/k_dx2_670k.md" if rf["traffic"] else "no capture of this kernel source"
     tail_ms = sum(prof[k][1] for k in prof if k.startswith("tail") or k in ("xt", "dx_reduce")) / args.steps
     tail_rf = roofline_of(work["tail"][0], work["tail"][1], tail_ms, peaks)
 
