@@ -614,8 +614,11 @@ size_t step_smem(int Bp, int k, int G) { return v2::step_layout(Bp, k, G).total;
 size_t dx_smem(int band, int k, int G, int ns) { return v2::dx_layout(band, k, G, ns).total; }
 
 // Band width and ring depth of the dX pass: the fewest bands whose accumulator
-// still leaves at least three stages (up to eight) in the shared memory left
-// after `reserve` bytes.  Returns false when even a band of 8 features does not fit.
+// still leaves at least two stages (up to eight) in the shared memory left after
+// `reserve` bytes.  Fewer bands mean fewer CTAs staging each group's dY tile and
+// weight block, which outweighs a deeper ring (measured at 8.6M labels: 3 bands
+// with 2 stages beat 4 bands with 3).  Returns false when even a band of 8
+// features does not fit.
 bool dx_config(int G, int k, int d, size_t smem_optin, size_t reserve, int* band, int* ns) {
   const v2::DxLayout one = v2::dx_layout(0, k, G, 1), none = v2::dx_layout(0, k, G, 0);
   const long stage = (long)one.total - (long)none.total;
@@ -623,7 +626,7 @@ bool dx_config(int G, int k, int d, size_t smem_optin, size_t reserve, int* band
     const int bw = ((d + nb - 1) / nb + 7) & ~7;
     const long left = (long)smem_optin - (long)reserve - (long)dx_smem(bw, k, G, 0);
     const long n = left / stage;
-    if (n >= 3 || (bw == 8 && n >= 2)) {
+    if (n >= 2) {
       *band = bw;
       *ns = (int)std::min<long>(n, v2::kMaxDxStages);
       return true;
