@@ -243,3 +243,57 @@ void ref_dx_at(int dt, const void* X, const void* W, const void* dY, const int32
     out[i] = acc;
   }
 }
+
+/* ---- two-stage top-k scoring ------------------------------------------------
+ * Source: "A Faster Generalized Two-Stage Approximate Top-K" (summary page),
+ * Methodology: stage 1 splits the N scores into buckets and keeps the top K' of
+ * each bucket; stage 2 returns the top K of the buckets' K' survivors (K' = K:
+ * the exact top K).  Here the scores of one sample are the logits of its L tail
+ * labels, and bucket j holds the labels of groups [j*n_g/nb, (j+1)*n_g/nb):
+ * contiguous whole groups (this project's reading; the page analyses random
+ * partitions).  Order: larger score first, equal scores by smaller label id.
+ * For each requested sample row rows[i]: out_val[i*K + j], out_id[i*K + j]. */
+static int ranks_before(double v1, int64_t i1, double v2, int64_t i2) {
+  return v1 > v2 || (v1 == v2 && i1 < i2);
+}
+/* insert (v, id) into the list (vals, ids) of length n, kept in rank order */
+static void keep_best(double* vals, int64_t* ids, int32_t n, double v, int64_t id) {
+  if (!ranks_before(v, id, vals[n - 1], ids[n - 1])) return;
+  int32_t j = n - 1;
+  while (j > 0 && ranks_before(v, id, vals[j - 1], ids[j - 1])) {
+    vals[j] = vals[j - 1];
+    ids[j] = ids[j - 1];
+    --j;
+  }
+  vals[j] = v;
+  ids[j] = id;
+}
+void ref_topk(int dt, const void* X, const void* W, const int32_t* idx, int32_t d, int64_t n_groups,
+              int32_t G, int32_t k, int32_t K, int32_t Kp, int32_t nb, int64_t n_rows, const int32_t* rows,
+              double* out_val, int64_t* out_id) {
+#pragma omp parallel for schedule(dynamic)
+  for (int64_t i = 0; i < n_rows; ++i) {
+    const int32_t b = rows[i];
+    double* cv = (double*)malloc(sizeof(double) * (size_t)nb * Kp);
+    int64_t* ci = (int64_t*)malloc(sizeof(int64_t) * (size_t)nb * Kp);
+    for (int32_t j = 0; j < nb; ++j) {           /* stage 1: top Kp of bucket j */
+      double* bv = cv + (size_t)j * Kp;
+      int64_t* bi = ci + (size_t)j * Kp;
+      for (int32_t e = 0; e < Kp; ++e) {
+        bv[e] = -INFINITY;
+        bi[e] = INT64_MAX;
+      }
+      const int64_t ga = (int64_t)j * n_groups / nb, gb = (int64_t)(j + 1) * n_groups / nb;
+      for (int64_t l = ga * G; l < gb * G; ++l) keep_best(bv, bi, Kp, logit_at(dt, X, W, idx, d, G, k, b, l), l);
+    }
+    double* ov = out_val + i * K;                  /* stage 2: top K of the survivors */
+    int64_t* oi = out_id + i * K;
+    for (int32_t e = 0; e < K; ++e) {
+      ov[e] = -INFINITY;
+      oi[e] = INT64_MAX;
+    }
+    for (int64_t c = 0; c < (int64_t)nb * Kp; ++c) keep_best(ov, oi, K, cv[c], ci[c]);
+    free(cv);
+    free(ci);
+  }
+}

@@ -62,6 +62,7 @@ def _load():
                                   P, P, D, I64, P, P, P]
         lib.ref_dx_at.argtypes = [ctypes.c_int, P, P, P, P, I32, I32, I64, I32, I32, ctypes.c_int,
                                   P, P, D, I64, P, P, P]
+        lib.ref_topk.argtypes = [ctypes.c_int, P, P, P, I32, I64, I32, I32, I32, I32, I32, I64, P, P, P]
         _lib = lib
     return _lib
 
@@ -199,6 +200,24 @@ def dx_at(X, W, idx, G, bs, fs, *, dY=None, pos=None, scale=1.0) -> np.ndarray:
                       G, idx.shape[1], int(fused), _ptr(rp), _ptr(ids), scale, len(bs),
                       _ptr(bs), _ptr(fs), _ptr(out))
     return out
+
+
+# ------------------------------------------------------- two-stage top-k scoring
+def topk(X, W, idx, G, K, Kp, n_buckets, rows=None) -> Tuple[np.ndarray, np.ndarray]:
+    """Two-stage top-K of the tail logits of the given sample rows ("A Faster
+    Generalized Two-Stage Approximate Top-K", Methodology): stage 1 keeps the top
+    Kp of each bucket, bucket j = the labels of groups [j*n_g/nb, (j+1)*n_g/nb);
+    stage 2 returns the top K of the survivors.  Order: larger logit first, equal
+    logits by smaller label id.  Returns (values float64 [n, K], ids int64 [n, K])."""
+    X, W, idx = _c(X), _c(W), _c(idx, np.int32)
+    B = X.shape[0]
+    rows = np.arange(B, dtype=np.int32) if rows is None else _c(rows, np.int32)
+    n_groups = idx.shape[0]
+    vals = np.empty((len(rows), K))
+    ids = np.empty((len(rows), K), dtype=np.int64)
+    _load().ref_topk(_dt(X), _ptr(X), _ptr(W), _ptr(idx), X.shape[1], n_groups, G, idx.shape[1], K, Kp,
+                     n_buckets, len(rows), _ptr(rows), _ptr(vals), _ptr(ids))
+    return vals, ids
 
 
 # ---------------------------------------------------------------- dense head

@@ -355,3 +355,65 @@ def test_input_generator_recipe():
         assert np.all(np.diff(r) > 0) and r.min() >= 0 and r.max() < 1000
     (hp, hi), (tp, ti) = I.split_head_tail(rp, ids, 100)
     assert hp[-1] + tp[-1] == len(ids) and (hi < 100).all() and (ti >= 0).all()
+
+
+# ------------------------------------------------------- two-stage top-k scoring
+# "A Faster Generalized Two-Stage Approximate Top-K" (summary page), Methodology:
+# stage 1 keeps the top K' of each bucket, stage 2 the top K of the survivors.
+def _exact_topk(z, K):
+    """Top K of each row by (larger value, smaller id): a full lexicographic sort."""
+    out_v, out_i = [], []
+    for row in z:
+        order = np.lexsort((np.arange(len(row)), -row))[:K]
+        out_v.append(row[order])
+        out_i.append(order)
+    return np.array(out_v), np.array(out_i)
+
+
+def _topk_case(seed=0, B=6, d=64, n_groups=40, G=16, k=8):
+    idx = I.make_idx(n_groups, k, d, seed)
+    X = I.make_normal((B, d), 1.0, seed, 1, "f32")
+    W = I.make_normal((n_groups * G, k), 1.0 / math.sqrt(k), seed, 2, "f32")
+    return idx, X, W, O.forward(X, W, idx, G)
+
+
+@pytest.mark.parametrize("K,nb", [(1, 1), (5, 7), (8, 40), (3, 13)])
+def test_topk_with_kp_equal_k_is_the_exact_top_k(K, nb):
+    idx, X, W, z = _topk_case()
+    v, i = O.topk(X, W, idx, 16, K, K, nb)
+    ev, ei = _exact_topk(z, K)
+    assert np.array_equal(i, ei) and np.allclose(v, ev, rtol=0, atol=1e-12)
+
+
+def test_topk_one_per_group_brute_force():
+    # nb = n_groups and K' = 1: the survivors are the group maxima
+    idx, X, W, z = _topk_case(seed=3)
+    G, K, n_groups = 16, 6, 40
+    v, i = O.topk(X, W, idx, G, K, 1, n_groups)
+    for r in range(z.shape[0]):
+        cand = []
+        for g in range(n_groups):
+            seg = z[r, g * G:(g + 1) * G]
+            j = int(np.lexsort((np.arange(G), -seg))[0])
+            cand.append((-seg[j], g * G + j))
+        best = sorted(cand)[:K]
+        assert [c[1] for c in best] == list(i[r]) and np.allclose([-c[0] for c in best], v[r], atol=1e-12)
+
+
+def test_topk_recall_grows_with_kp_and_survivors_are_true_scores():
+    idx, X, W, z = _topk_case(seed=5, B=8, n_groups=64)
+    K, nb = 8, 4
+    ev, ei = _exact_topk(z, K)
+    prev = -1.0
+    for Kp in (1, 2, 4, 8):
+        v, i = O.topk(X, W, idx, 16, K, Kp, nb, rows=np.arange(8))
+        # every returned entry is a real (label, logit) pair, ids distinct, ranked
+        for r in range(8):
+            ok = i[r] < 2**62
+            assert np.allclose(v[r][ok], z[r, i[r][ok]], atol=1e-12)
+            assert len(set(i[r][ok].tolist())) == ok.sum()
+            assert np.all(np.diff(v[r][ok]) <= 0)
+        recall = np.mean([len(set(i[r].tolist()) & set(ei[r].tolist())) / K for r in range(8)])
+        assert recall >= prev
+        prev = recall
+    assert prev == 1.0
