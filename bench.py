@@ -282,6 +282,33 @@ def timed(fn, steps, warmup, dist):
     return ms
 
 
+def infer_topk(run, steps, warmup, peaks, K=5, kp=4):
+    """Inference scoring at the same workload: the top-K tail labels per sample by
+    the two-stage top-k (the top kp of each of n_buckets buckets of whole groups,
+    then the top K of the survivors), device-timed; logits never reach memory.
+    With one bucket per SM and kp = 4, a top-5 label is missed only when all five
+    share one bucket."""
+    import torch
+    H, wl = run.H, run.wl
+    nb = min(wl.n_groups, torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count)
+    ws = torch.empty(H.haste_topk_workspace_size(run.plan, wl.B, H.HASTE_BF16, nb, kp), dtype=torch.uint8,
+                     device="cuda")
+    ov = torch.empty((wl.B, K), dtype=torch.float32, device="cuda")
+    oi = torch.empty((wl.B, K), dtype=torch.int32, device="cuda")
+    fn = lambda: H.haste_topk(run.plan, run.X, run.W, K, kp, nb, ov, oi, ws)
+    H.haste_profile_start()
+    ms = timed(fn, steps, warmup, False)
+    prof = H.haste_profile_stop()
+    n_l, t_ms = prof.get("topk_score", (1, ms))
+    flops = 2.0 * wl.B * wl.L * wl.k
+    nbytes = wl.L * wl.k * 2 + 4 * wl.n_groups * wl.k + wl.B * wl.d * 2
+    rf = roofline_of(flops, nbytes, t_ms / max(n_l, 1), peaks)
+    rf["kernel"] = "topk_score"
+    return {"metric": f"top-{K} tail scoring samples/s", "value": round(wl.B * steps / (ms / 1e3), 1),
+            "ms_per_call": round(ms / steps, 4), "k": K, "kp": kp, "n_buckets": nb, "exact": kp >= K,
+            "roofline": rf}
+
+
 # ----------------------------------------------------------- CPU baseline
 def oracle_step_seconds(inp, n_sub_groups):
     """Oracle time of one step on the first n_sub_groups groups (tail) plus the
@@ -422,6 +449,8 @@ def main():
     run.e2e_setup()
     ms_e2e = timed(run.e2e_step, args.steps, args.warmup, dist)
 
+    inference = infer_topk(run, args.steps, args.warmup, peaks) if wl.dtype == "bf16" and wl.B <= 256 else None
+
     launches = sum(n for n, _ in prof.values())
     work = algorithmic(wl)
     dom = max((k for k in prof if k in work), key=lambda k: prof[k][1])
@@ -452,6 +481,7 @@ def main():
         "gpu_launches": launches,
         "clocks": clocks,
         "plan_build_s": round(run.plan_s, 3),
+        "inference": inference,
         "index_bytes": run.plan.info()[0],
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -193,6 +193,33 @@ haste_status_t haste_bce_step(haste_plan_t plan, int32_t B, haste_dtype_t dtype,
                               haste_targets_t tail_pos, float grad_scale, float* loss, void* dW, float* dX,
                               int accumulate, void* ws, size_t ws_bytes, haste_stream_t stream);
 
+/* ----------------------------------------------------- top-k scoring --- */
+
+/* Workspace bytes of haste_topk at (B, n_buckets, kp). */
+size_t haste_topk_workspace_size(haste_plan_t plan, int32_t B, haste_dtype_t dtype, int32_t n_buckets, int32_t kp);
+
+/* Two-stage top-k scoring of the tail logits, for inference (P@k).
+ * Scores: logits[b, l] = X[b, I_g] . W[l, :] as haste_forward (Methodology 1 of
+ * the HASTE summary page); they are ranked inside the forward epilogue and never
+ * written to memory.  Selection: "A Faster Generalized Two-Stage Approximate
+ * Top-K" (summary page, Methodology): stage 1 splits the labels into n_buckets
+ * buckets of whole groups, bucket j = the labels of groups
+ * [j*n_groups/n_buckets, (j+1)*n_groups/n_buckets), and keeps the kp best logits
+ * of each bucket per sample; stage 2 returns the k best of the n_buckets*kp
+ * survivors.  kp = k gives the exact top k; kp < k may miss labels that share a
+ * bucket with kp better ones.  Rank order: larger logit first, equal logits by
+ * smaller label id.
+ *   X        device [B, d] bf16;  W device [L, k] bf16
+ *   out_val  device [B, k] fp32, rank order;  out_id device [B, k] int32 tail ids
+ * Supported: bf16, G in {16, 32, 64}, k of the plan in {64, 128}, B <= 256,
+ * kp in {1, 2, 4, 8}, 1 <= n_buckets <= n_groups, 1 <= k <= min(64, n_buckets*kp).
+ * Other arguments return HASTE_ERR_INVALID_ARG or HASTE_ERR_UNSUPPORTED_SHAPE.
+ * Stage 1 runs one CTA per bucket (n_buckets = the number of SMs uses the whole
+ * GPU).  The dense head's logits are not included. */
+haste_status_t haste_topk(haste_plan_t plan, int32_t B, haste_dtype_t dtype, const void* X, const void* W,
+                          int32_t k, int32_t kp, int32_t n_buckets, float* out_val, int32_t* out_id, void* ws,
+                          size_t ws_bytes, haste_stream_t stream);
+
 /* -------------------------------------------------------------- dense head --- */
 
 /* Workspace bytes of the head calls at (B, H, d). */

@@ -19,6 +19,7 @@
 #include "head.cu"
 #include "tail.cu"
 #include "tail_v2.cu"
+#include "topk.cu"
 
 using namespace haste;
 
@@ -707,6 +708,68 @@ haste_status_t check_head(int B, int H, int d, haste_dtype_t dt) {
   return HASTE_OK;
 }
 }  // namespace
+
+// Workspace of haste_topk: X^T [d, Bp] (input dtype) and the stage-1 candidates
+// [n_buckets][Bp][kp] (fp32 values, int32 label ids).
+static size_t topk_ws(const haste_plan_s& p, int B, int E, int n_buckets, int kp, size_t* cand) {
+  const int Bp = round_up(B, 128);
+  *cand = align256((size_t)p.d * Bp * E);
+  return *cand + align256((size_t)n_buckets * Bp * kp * 8);
+}
+
+size_t haste_topk_workspace_size(haste_plan_t p, int32_t B, haste_dtype_t dt, int32_t n_buckets, int32_t kp) {
+  if (!p || B <= 0 || n_buckets <= 0 || kp <= 0) return 0;
+  size_t cand;
+  return topk_ws(*p, B, elem_bytes(dt), n_buckets, kp, &cand);
+}
+
+haste_status_t haste_topk(haste_plan_t p, int32_t B, haste_dtype_t dt, const void* X, const void* W, int32_t k,
+                          int32_t kp, int32_t n_buckets, float* out_val, int32_t* out_id, void* ws, size_t ws_bytes,
+                          haste_stream_t stream) {
+  DeviceInfo di;
+  haste_status_t st = device_info(di);
+  if (st == HASTE_OK) st = check_tail(p, B, dt, di);
+  if (st != HASTE_OK) return st;
+  if (!X || !W || !out_val || !out_id) return fail(HASTE_ERR_INVALID_ARG, "NULL pointer");
+  const int Bp = round_up(B, 128);
+  if (dt != HASTE_BF16 || !topk_host::supported(p->G, p->k, Bp, kp))
+    return fail(HASTE_ERR_UNSUPPORTED_SHAPE,
+                "top-k scoring needs bf16, G in {16,32,64}, k in {64,128}, B <= 256, kp in {1,2,4,8}");
+  if (n_buckets < 1 || (int64_t)n_buckets > p->n_groups)
+    return fail(HASTE_ERR_INVALID_ARG, "n_buckets=%d must lie in [1, n_groups]", n_buckets);
+  if (k < 1 || k > 64 || (int64_t)k > (int64_t)n_buckets * kp)
+    return fail(HASTE_ERR_INVALID_ARG, "k=%d must lie in [1, min(64, n_buckets * kp)]", k);
+  if ((size_t)n_buckets * kp * 8 > (size_t)di.smem_optin - 1024)
+    return fail(HASTE_ERR_UNSUPPORTED_SHAPE, "n_buckets * kp candidates exceed shared memory");
+  if (topk_host::smem_stage1(Bp, p->k, p->G, kp) > (size_t)di.smem_optin)
+    return fail(HASTE_ERR_UNSUPPORTED_SHAPE, "top-k tiles exceed shared memory");
+  size_t cand;
+  const size_t need = topk_ws(*p, B, 2, n_buckets, kp, &cand);
+  if ((st = check_ws(ws, ws_bytes, need)) != HASTE_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* wb = static_cast<uint8_t*>(ws);
+  TailArgs xa = make_args(*p, B);
+  xa.Xt = wb;
+  topk::Args a{};
+  a.sh = xa.sh;
+  a.idx = p->idx_d;
+  a.cand_val = reinterpret_cast<float*>(wb + cand);
+  a.cand_id = reinterpret_cast<int32_t*>(wb + cand + (size_t)n_buckets * Bp * kp * 4);
+  cudaError_t e;
+  {
+    ProfScope ps("xt", s);
+    e = xt<__nv_bfloat16>(xa, X, wb, s);
+  }
+  if (e == cudaSuccess) {
+    ProfScope ps("topk_score", s);
+    e = topk_host::launch_stage1(p->G, p->k, kp, a, n_buckets, wb, W, s);
+  }
+  if (e == cudaSuccess) {
+    ProfScope ps("topk_merge", s);
+    e = topk_host::launch_stage2(a.cand_val, a.cand_id, B, Bp, n_buckets, kp, k, out_val, out_id, s);
+  }
+  return e == cudaSuccess ? HASTE_OK : cuda_fail(e, "haste_topk launch");
+}
 
 size_t haste_head_workspace_size(int32_t B, int32_t H, int32_t d, haste_dtype_t dt) {
   if (B <= 0 || H <= 0 || d <= 0) return 0;

@@ -77,6 +77,8 @@ def lib() -> ctypes.CDLL:
         "haste_backward_dx": ([P, I32, S, P, P, P, S, P, SZ, P], S),
         "haste_backward_dx_noalloc": ([P, I32, S, P, P, P, S, P], S),
         "haste_bce_step": ([P, I32, S, P, P, Targets, F, P, P, P, S, P, SZ, P], S),
+        "haste_topk_workspace_size": ([P, I32, S, I32, I32], SZ),
+        "haste_topk": ([P, I32, S, P, P, I32, I32, I32, P, P, P, SZ, P], S),
         "haste_head_workspace_size": ([I32, I32, I32, S], SZ),
         "haste_head_forward": ([I32, I32, I32, S, P, P, P, P, F, P, P, SZ, P], S),
         "haste_head_backward": ([I32, I32, I32, S, P, P, P, P, P, P, SZ, P], S),
@@ -232,6 +234,19 @@ def haste_bce_step(plan: Plan, X, W, pos_row_ptr, pos_ids, grad_scale: float, lo
     _check(lib().haste_bce_step(plan.handle, X.shape[0], dtype_code(X), _tptr(X), _tptr(W), tg, float(grad_scale),
                                 _tptr(loss), _tptr(dW), _tptr(dX), int(accumulate), p, n, _stream(stream)),
            "haste_bce_step")
+
+
+# ------------------------------------------------------------ top-k scoring
+def haste_topk_workspace_size(plan: Plan, B: int, dtype: int, n_buckets: int, kp: int) -> int:
+    return int(lib().haste_topk_workspace_size(plan.handle, B, dtype, n_buckets, kp))
+
+
+def haste_topk(plan: Plan, X, W, k: int, kp: int, n_buckets: int, out_val, out_id, ws, stream=None) -> None:
+    """Two-stage top-k of the tail logits per sample (see include/haste.h):
+    out_val [B, k] fp32 and out_id [B, k] int32, larger logit first."""
+    p, n = _ws(ws)
+    _check(lib().haste_topk(plan.handle, X.shape[0], dtype_code(X), _tptr(X), _tptr(W), int(k), int(kp),
+                            int(n_buckets), _tptr(out_val), _tptr(out_id), p, n, _stream(stream)), "haste_topk")
 
 
 # ---------------------------------------------------------------- dense head

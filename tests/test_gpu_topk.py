@@ -1,0 +1,115 @@
+"""GPU parity of the two-stage top-k scoring (haste_topk) against the fp64 oracle.
+
+Stage 1 keeps the top kp logits of each bucket of whole groups inside the forward
+epilogue, stage 2 the top k of the survivors ("A Faster Generalized Two-Stage
+Approximate Top-K", summary page, Methodology; scores: HASTE Methodology 1).
+The GPU ranks fp32 logits of bf16 inputs and the oracle fp64 logits of the same
+values, so labels whose logits differ by less than the rounding may trade ranks:
+the checks compare what is unique (the value at every rank, every returned id's
+true logit, distinct ids) and require identical ids wherever the oracle's ranking
+has no near-tie.
+"""
+import math
+
+import numpy as np
+import pytest
+
+from oracle import oracle as O
+from structured_sparse_output_b200 import haste as H
+from structured_sparse_output_b200 import inputs as I
+from tests.helpers import to_torch
+
+pytestmark = pytest.mark.gpu
+torch = pytest.importorskip("torch")
+
+TOL = 2e-4  # |fp32 - fp64| of a k-term bf16 dot product is ~1e-6; generous margin
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _need_gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    H.lib()
+    yield
+    torch.cuda.synchronize()
+    assert H.haste_device_status() == H.HASTE_OK
+
+
+def _run(plan, X, W, K, kp, nb):
+    B = X.shape[0]
+    ws = torch.empty(H.haste_topk_workspace_size(plan, B, H.HASTE_BF16, nb, kp), dtype=torch.uint8, device="cuda")
+    ov = torch.full((B, K), float("nan"), device="cuda")
+    oi = torch.full((B, K), -1, dtype=torch.int32, device="cuda")
+    H.haste_topk(plan, X, W, K, kp, nb, ov, oi, ws)
+    torch.cuda.synchronize()
+    return ov.cpu().numpy().astype(np.float64), oi.cpu().numpy().astype(np.int64)
+
+
+def _check(gv, gi, rv, ri, true_logit, L, what):
+    K = gv.shape[1]
+    for r in range(gv.shape[0]):
+        assert len(set(gi[r].tolist())) == K and gi[r].min() >= 0 and gi[r].max() < L, what
+        assert np.all(np.diff(gv[r]) <= 0), what                       # rank order
+        assert np.allclose(gv[r], true_logit(r, gi[r]), atol=TOL), what  # true (label, logit) pairs
+        assert np.allclose(gv[r], rv[r], atol=TOL), what                 # same value at every rank
+        gaps = np.abs(np.diff(rv[r]))
+        clear = np.ones(K, bool)
+        clear[:-1] &= gaps > TOL
+        clear[1:] &= gaps > TOL
+        assert np.array_equal(gi[r][clear], ri[r][clear]), what
+
+
+CASES = [
+    dict(B=130, d=256, n_groups=300, G=32, k=64, K=8, kp=8, nb=37),   # exact, ragged batch
+    dict(B=64, d=320, n_groups=97, G=16, k=64, K=5, kp=8, nb=1),      # one bucket
+    dict(B=256, d=768, n_groups=200, G=64, k=128, K=16, kp=4, nb=50),  # approximate (kp < K)
+    dict(B=200, d=512, n_groups=150, G=32, k=128, K=3, kp=1, nb=150),  # one bucket per group
+    dict(B=32, d=256, n_groups=64, G=16, k=64, K=64, kp=8, nb=8),      # k = n_buckets * kp
+]
+
+
+@pytest.mark.parametrize("c", CASES, ids=lambda c: "B{B}_G{G}_k{k}_K{K}_kp{kp}_nb{nb}".format(**c))
+def test_topk_matches_oracle(c):
+    B, d, n_groups, G, k = c["B"], c["d"], c["n_groups"], c["G"], c["k"]
+    idx = I.make_idx(n_groups, k, d, 0)
+    X = I.make_normal((B, d), 1.0, 0, 1, "bf16")
+    W = I.make_normal((n_groups * G, k), 1.0 / math.sqrt(k), 0, 2, "bf16")
+    plan = H.haste_plan(idx, G, d)
+    gv, gi = _run(plan, to_torch(X), to_torch(W), c["K"], c["kp"], c["nb"])
+    rv, ri = O.topk(X, W, idx, G, c["K"], c["kp"], c["nb"])
+    z = O.forward(X, W, idx, G)
+    _check(gv, gi, rv, ri, lambda r, ids: z[r, ids], n_groups * G, str(c))
+    # bitwise run-to-run determinism
+    gv2, gi2 = _run(plan, to_torch(X), to_torch(W), c["K"], c["kp"], c["nb"])
+    assert np.array_equal(gi, gi2) and np.array_equal(gv, gv2)
+
+
+def test_topk_full_size_670k_sampled_rows():
+    wl = I.WORKLOADS["670k"]
+    idx = I.make_idx(wl.n_groups, wl.k, wl.d, 0)
+    X = I.make_normal((wl.B, wl.d), 1.0, 0, 1, "bf16")
+    W = I.make_normal((wl.L, wl.k), 1.0 / math.sqrt(wl.k), 0, 2, "bf16")
+    plan = H.haste_plan(idx, wl.G, wl.d)
+    nb = torch.cuda.get_device_properties(0).multi_processor_count
+    gv, gi = _run(plan, to_torch(X), to_torch(W), 5, 8, nb)
+    rows = np.array([0, 1, 77, wl.B - 1], dtype=np.int32)
+    rv, ri = O.topk(X, W, idx, wl.G, 5, 8, nb, rows=rows)
+    true = lambda r, ids: O.logits_at(X, W, idx, wl.G, np.full(len(ids), rows[r], np.int32), ids.astype(np.int64))
+    _check(gv[rows], gi[rows], rv, ri, true, wl.L, "670k")
+
+
+def test_topk_argument_errors():
+    idx = I.make_idx(40, 64, 256, 0)
+    plan = H.haste_plan(idx, 32, 256)
+    X = torch.zeros((8, 256), dtype=torch.bfloat16, device="cuda")
+    W = torch.zeros((40 * 32, 64), dtype=torch.bfloat16, device="cuda")
+    ov = torch.empty((8, 4), device="cuda")
+    oi = torch.empty((8, 4), dtype=torch.int32, device="cuda")
+    ws = torch.empty(H.haste_topk_workspace_size(plan, 8, H.HASTE_BF16, 4, 2), dtype=torch.uint8, device="cuda")
+    for K, kp, nb, code in ((4, 3, 4, H.HASTE_ERR_UNSUPPORTED_SHAPE),   # kp not a power of two <= 8
+                            (9, 2, 4, H.HASTE_ERR_INVALID_ARG),         # k > n_buckets * kp
+                            (4, 2, 0, H.HASTE_ERR_INVALID_ARG),         # no bucket
+                            (4, 2, 41, H.HASTE_ERR_INVALID_ARG)):       # more buckets than groups
+        with pytest.raises(H.HasteError) as e:
+            H.haste_topk(plan, X, W, K, kp, nb, ov, oi, ws)
+        assert e.value.status == code
