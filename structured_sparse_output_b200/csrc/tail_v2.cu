@@ -571,16 +571,25 @@ __global__ void __launch_bounds__(kDxThreads, 1)
       // the team finishes group i-1 before any of its warps adds group i
       named_bar(1 + hb, 128);
       if (ok && act) {
+        // loads ahead of stores: the chunks are distinct, but the compiler cannot
+        // see that and would otherwise order each load after the previous chunk's
+        // store (eight shared-memory round trips in a row)
         uint8_t* row = acc + (uint32_t)f * 512u;
 #pragma unroll
-        for (int cq = 0; cq < 8; ++cq) {
-          float4* p = reinterpret_cast<float4*>(row + (uint32_t)(((8 * hb + cq) ^ (f & 7)) * 16));
-          float4 o = *p;
-          o.x += v[4 * cq];
-          o.y += v[4 * cq + 1];
-          o.z += v[4 * cq + 2];
-          o.w += v[4 * cq + 3];
-          *p = o;
+        for (int h4 = 0; h4 < 8; h4 += 4) {  // two batches of four chunks (register budget)
+          float4 o[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            o[e] = *reinterpret_cast<const float4*>(row + (uint32_t)(((8 * hb + h4 + e) ^ (f & 7)) * 16));
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int cq = h4 + e;
+            o[e].x += v[4 * cq];
+            o[e].y += v[4 * cq + 1];
+            o[e].z += v[4 * cq + 2];
+            o[e].w += v[4 * cq + 3];
+            *reinterpret_cast<float4*>(row + (uint32_t)(((8 * hb + cq) ^ (f & 7)) * 16)) = o[e];
+          }
         }
       }
     }
