@@ -12,14 +12,13 @@
 //              shared memory for the dW product and to the group-major gradient
 //              buffer of the dX pass), then dW is read out of TMEM.
 // k_dx2 -- dX pass: per CTA (128-row batch tile, feature band, group chunk):
-//   warps 0-3 stage the dY tile and the weight columns of the band's slots into
-//   a shared-memory ring whose stages publish themselves when their copies land
-//   (warp 0 also writes the slot metadata into a 16-entry ring), warp 4 issues
-//   Z = dY_g . W_g[:, slots] into one of four TMEM buffers, warps 5-20 add the
-//   columns of Z into a fp32 band accumulator in shared memory.
-//   Scatter warp (q, p) owns batch rows [32q, 32q+32) and the p-th quarter of the
-//   band's features, so every feature receives its group terms in ascending
-//   group order, deterministically.
+//   warp 0 (one thread) loads each group's dY tile and G x k weight block into a
+//   shared-memory ring with TMA, warp 1 issues Z^T = W_g^T . dY_g^T (TMEM lane =
+//   slot, column = batch row) into one of four TMEM buffers, and warps 2-17 add
+//   the Z^T rows of the slots whose features fall in the band into a fp32 band
+//   accumulator in shared memory.  A team of four warps (one per TMEM lane
+//   quarter) owns a batch quarter and finishes a group before the next, so every
+//   feature receives its group terms in ascending group order, deterministically.
 #include "tail.cuh"
 
 namespace haste {
@@ -47,8 +46,6 @@ struct DxArgs {
   int dy_xg, dy_yg;
 };
 
-constexpr int kMetaSlots = 16;  // metadata ring of the dX pass (twice the deepest data ring)
-constexpr int kMetaHdr = 8;    // 5 slot split points, s0, N, 1 spare
 
 constexpr int kMaxDxStages = 8;  // deepest data ring of the dX pass
 
@@ -72,18 +69,17 @@ __host__ __device__ inline StepLayout step_layout(int Bp, int k, int G) {
 }
 
 struct DxLayout {
-  uint32_t dy, w, acc, meta, bars, total, dy_stride, w_stride, meta_stride;
+  uint32_t dy, w, acc, bars, total, dy_stride, w_stride;
 };
-// Shared memory of the dX pass: ns stages of (dY tile, weight columns), the fp32
-// band accumulator [band][128], the metadata ring and the barriers.
+// Shared memory of the dX pass: ns stages of (dY tile, weight block), the fp32
+// band accumulator [band][128] and the barriers.
 __host__ __device__ inline DxLayout dx_layout(int band, int k, int G, int ns) {
   DxLayout L;
   L.dy_stride = (uint32_t)((128 * G * 2 + 1023) & ~1023);
-  // 64-slot blocks of weight columns: rows [s0, hi) of Z^T need two blocks only
-  // when k = 128 (hi - s0 <= k); with k = 64 the second block the MMA reads is the
-  // next region of shared memory and feeds only TMEM lanes no thread reads.
+  // 64-slot blocks of the weight block: Z^T has 128 slot rows; with k = 64 the
+  // second block the MMA reads is the next region of shared memory and feeds only
+  // TMEM lanes (slots >= k) that no thread reads.
   L.w_stride = (uint32_t)((k / 64) * G * 128);
-  L.meta_stride = 0;
   uint32_t off = 0;
   L.dy = off;
   off += ns * L.dy_stride;
@@ -91,8 +87,6 @@ __host__ __device__ inline DxLayout dx_layout(int band, int k, int G, int ns) {
   off += ns * L.w_stride;
   L.acc = off;
   off += (uint32_t)band * 128 * 4;
-  L.meta = off;
-  off += kMetaSlots * L.meta_stride;
   off = (off + 7) & ~7u;
   L.bars = off;
   off += 512;
