@@ -155,14 +155,17 @@ __global__ void __launch_bounds__(kGThreads, 1) k_gemm(GemmArgs a) {
       tmem_wait_ld();
       if (m >= a.M) continue;
       const int n = n0 + c;
-      if constexpr (kEpi == kEpiPartial) {
-        float* dst = static_cast<float*>(a.C) + ((int64_t)split * a.M + m) * a.N + n;
-        for (int i = 0; i < 16; ++i)
-          if (n + i < a.N) dst[i] = v[i];
-      } else if constexpr (kEpi == kEpiStoreF32) {
-        float* dst = static_cast<float*>(a.C) + (int64_t)m * a.ldc + n;
-        for (int i = 0; i < 16; ++i)
-          if (n + i < a.N) dst[i] = v[i];
+      if constexpr (kEpi == kEpiPartial || kEpi == kEpiStoreF32) {
+        float* dst = kEpi == kEpiPartial ? static_cast<float*>(a.C) + ((int64_t)split * a.M + m) * a.N + n
+                                         : static_cast<float*>(a.C) + (int64_t)m * a.ldc + n;
+        const int64_t ld = kEpi == kEpiPartial ? a.N : a.ldc;
+        if (n + 16 <= a.N && (ld & 3) == 0 && (reinterpret_cast<uintptr_t>(a.C) & 15) == 0) {  // 4 x 16 B
+#pragma unroll
+          for (int i = 0; i < 16; i += 4) *reinterpret_cast<float4*>(dst + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+        } else {
+          for (int i = 0; i < 16; ++i)
+            if (n + i < a.N) dst[i] = v[i];
+        }
       } else {
         if constexpr (kEpi == kEpiBce) {
           float lin = 0.f, prod = 1.f;
@@ -180,8 +183,17 @@ __global__ void __launch_bounds__(kGThreads, 1) k_gemm(GemmArgs a) {
           loss_acc += lin - __logf(prod);
         }
         T* dst = static_cast<T*>(a.C) + (int64_t)m * a.ldc + n;
-        for (int i = 0; i < 16; ++i)
-          if (n + i < a.N) dst[i] = Elem<T>::from_f(v[i]);
+        if (sizeof(T) == 2 && n + 16 <= a.N && (a.ldc & 7) == 0 &&
+            (reinterpret_cast<uintptr_t>(a.C) & 15) == 0) {  // 2 x 16 B
+#pragma unroll
+          for (int i = 0; i < 16; i += 8)
+            *reinterpret_cast<uint4*>(dst + i) =
+                make_uint4(pack_bf16x2(v[i], v[i + 1]), pack_bf16x2(v[i + 2], v[i + 3]),
+                           pack_bf16x2(v[i + 4], v[i + 5]), pack_bf16x2(v[i + 6], v[i + 7]));
+        } else {
+          for (int i = 0; i < 16; ++i)
+            if (n + i < a.N) dst[i] = Elem<T>::from_f(v[i]);
+        }
       }
     }
   }

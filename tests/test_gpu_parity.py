@@ -157,6 +157,8 @@ HEAD_CASES = [
     dict(B=256, Hh=384, d=192, dtype="bf16"),
     dict(B=128, Hh=256, d=128, dtype="f32"),
     dict(B=256, Hh=4096, d=768, dtype="bf16"),
+    dict(B=100, Hh=200, d=136, dtype="bf16"),   # ragged: last 8 columns of every output tile, partial M tile
+    dict(B=70, Hh=100, d=36, dtype="f32"),
 ]
 
 
