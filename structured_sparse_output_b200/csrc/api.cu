@@ -122,9 +122,10 @@ class ProfScope {
   cudaEvent_t a_ = nullptr;
 };
 
-// Tiling of the dX pass: feature bands sized so the fp32 band accumulator fits
-// in shared memory next to the W and dY tiles (ns stages of them in the
-// pipelined kernel); group chunks so that all CTAs are resident.
+// Tiling of the dX pass: feature bands (at most 256 features, the MMA N, in the
+// pipelined kernel; sized so the fp32 band accumulator fits in shared memory in
+// the staged one); group chunks so that all CTAs are resident.  ns > 0: the
+// pipelined kernel with an ns-stage ring; ns = 0: the staged kernel.
 struct DxTiling {
   int band, n_bands, n_chunks, ns;
 };
@@ -137,19 +138,21 @@ bool use_v2(const haste_plan_s& p, int Bp, int elem) { return elem == 2 && tail2
 DxTiling dx_tiling(const haste_plan_s& p, int Bp, int elem, int sms, int smem_optin) {
   DxTiling t{};
   const int kHeadroom = 4096;  // static shared memory and launch reserve
-  int band = 8;
-  if (use_v2(p, Bp, elem)) {
-    if (!tail2::dx_config(p.G, p.k, p.d, (size_t)smem_optin, kHeadroom, &band, &t.ns)) t.ns = 2;
+  int per_chunk;
+  if (use_v2(p, Bp, elem) &&
+      tail2::dx_config(p.G, p.k, p.d, Bp, (size_t)smem_optin, kHeadroom, &t.band, &t.n_bands, &t.ns)) {
+    per_chunk = t.n_bands;  // a CTA covers every batch row of its band
   } else {
     const long avail = (long)smem_optin - (long)tail::smem_dx(elem, p.k, p.G, 0) - kHeadroom;
-    band = (int)std::min<long>(256, avail / 512);
+    int band = (int)std::min<long>(256, avail / 512);
+    band = std::max(8, band & ~7);
+    if (band > p.d) band = round_up(p.d, 8);
+    // as few bands as fit, then split d evenly between them
+    t.n_bands = (p.d + band - 1) / band;
+    t.band = round_up((p.d + t.n_bands - 1) / t.n_bands, 8);
+    t.ns = 0;
+    per_chunk = (Bp / 128) * t.n_bands;
   }
-  band = std::max(8, band & ~7);
-  if (band > p.d) band = round_up(p.d, 8);
-  // as few bands as fit, then split d evenly between them
-  t.n_bands = (p.d + band - 1) / band;
-  t.band = round_up((p.d + t.n_bands - 1) / t.n_bands, 8);
-  const int per_chunk = (Bp / 128) * t.n_bands;
   int c = std::max(1, sms / per_chunk);
   if ((int64_t)c > p.n_groups) c = (int)p.n_groups;
   t.n_chunks = c;
@@ -551,7 +554,7 @@ haste_status_t haste_backward_dx(haste_plan_t p, int32_t B, haste_dtype_t dt, co
   cudaError_t e;
   {
     ProfScope ps("tail_dx", s);
-    if (use_v2(*p, a.sh.Bp, E))
+    if (t.ns > 0)
       e = dx_v2(*p, B, W, dY, p->G, a.sh.L, a.dX_part, t, s);
     else
       e = dt == HASTE_BF16 ? tail::launch_backward_dx<__nv_bfloat16>(a, false, s)
@@ -596,7 +599,7 @@ haste_status_t haste_backward_dx_noalloc(haste_plan_t p, int32_t B, haste_dtype_
   a.band = t.band;
   a.n_bands = t.n_bands;
   a.n_chunks = t.n_chunks;
-  cudaError_t e = use_v2(*p, Bp, E) ? dx_v2(*p, B, W, dY, p->G, a.sh.L, a.dX_part, t, s)
+  cudaError_t e = t.ns > 0 ? dx_v2(*p, B, W, dY, p->G, a.sh.L, a.dX_part, t, s)
                  : dt == HASTE_BF16  ? tail::launch_backward_dx<__nv_bfloat16>(a, false, s)
                                      : tail::launch_backward_dx<float>(a, false, s);
   if (e == cudaSuccess) e = tail::launch_dx_reduce(a.dX_part, dX, t.n_chunks, p->d, Bp, B, accumulate, s);
@@ -635,7 +638,7 @@ haste_status_t haste_bce_step(haste_plan_t p, int32_t B, haste_dtype_t dt, const
   a.band = t.band;
   a.n_bands = t.n_bands;
   a.n_chunks = t.n_chunks;
-  const bool v2p = use_v2(*p, Bp, E) && tail2::step_smem(Bp, p->k, p->G) <= (size_t)di.smem_optin;
+  const bool v2p = use_v2(*p, Bp, E) && tail2::step_smem(Bp, p->k, p->G) <= (size_t)di.smem_optin && t.ns > 0;
   const int grid = v2p ? (int)std::min<int64_t>(p->n_groups, di.sms)
                        : dt == HASTE_BF16 ? tail::step_grid<__nv_bfloat16>(a, di.sms) : tail::step_grid<float>(a, di.sms);
   if (grid <= 0 || grid > kMaxLossParts) return fail(HASTE_ERR_CUDA, "could not size the fused step grid");
@@ -666,7 +669,7 @@ haste_status_t haste_bce_step(haste_plan_t p, int32_t B, haste_dtype_t dt, const
     ProfScope ps("tail_dx", s);
     if (v2p)
       e = dx_v2(*p, B, W, a.dY_out, (int64_t)Bp * p->G, p->G, a.dX_part, t, s);
-    else if (use_v2(*p, Bp, E))
+    else if (t.ns > 0)
       e = dx_v2(*p, B, W, a.dY_out, p->G, a.sh.L, a.dX_part, t, s);
     else
       e = dt == HASTE_BF16 ? tail::launch_backward_dx<__nv_bfloat16>(a, true, s)
