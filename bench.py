@@ -78,24 +78,34 @@ def algorithmic(wl):
     return out
 
 
-# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) of the
-# dominant kernel from one ncu capture (summaries under profiles/), valid only for
-# the kernel source they were taken on: (config, kernel) -> (bytes, source digest).
-TRAFFIC = {
-    ("670k", "tail_dx"): (529.1e6, "356b7444165b55d2"),
-}
-KERNEL_SOURCE = os.path.join(ROOT, "structured_sparse_output_b200", "csrc", "tail_v2.cu")
+# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) of a
+# kernel from one ncu capture (summaries under profiles/), valid only for the
+# source file it was taken on: (config, timed region) -> (bytes, source digest).
+TRAFFIC = {}
+# timed region -> (source file under csrc/, kernel name in the ncu summaries)
+KERNELS = {"tail_step": ("tail_v2.cu", "k_step2"), "tail_dx": ("dx_band.cu", "k_dx_band"),
+           "topk_score": ("topk.cu", "k_topk")}
+CSRC = os.path.join(ROOT, "structured_sparse_output_b200", "csrc")
+
+
+def source_digest(kernel):
+    import hashlib
+    src = os.path.join(CSRC, KERNELS[kernel][0])
+    if not os.path.exists(src):
+        return None
+    with open(src, "rb") as fh:
+        return hashlib.sha256(fh.read()).hexdigest()[:16]
 
 
 def traffic_of(config, kernel):
-    """The captured traffic, or None when the kernel source changed since the capture."""
-    import hashlib
+    """(bytes, where from): the captured traffic, or None when the kernel's source
+    changed since the capture (or it was never captured)."""
     got = TRAFFIC.get((config, kernel))
-    if got is None or not os.path.exists(KERNEL_SOURCE):
-        return None
-    with open(KERNEL_SOURCE, "rb") as fh:
-        digest = hashlib.sha256(fh.read()).hexdigest()[:16]
-    return got[0] if digest == got[1] else None
+    if got is None or kernel not in KERNELS:
+        return None, "no capture of this kernel"
+    if source_digest(kernel) != got[1]:
+        return None, "kernel source changed since the capture"
+    return got[0], f"ncu capture, profiles/{KERNELS[kernel][1]}_{config}.md"
 
 
 def roofline_of(flops, nbytes, ms, peaks, sustained=True):
@@ -304,6 +314,7 @@ def infer_topk(run, steps, warmup, peaks, K=5, kp=4):
     nbytes = wl.L * wl.k * 2 + 4 * wl.n_groups * wl.k + wl.B * wl.d * 2
     rf = roofline_of(flops, nbytes, t_ms / max(n_l, 1), peaks)
     rf["kernel"] = "topk_score"
+    rf["traffic"], rf["traffic_src"] = traffic_of(wl.name, "topk_score")
     return {"metric": f"top-{K} tail scoring samples/s", "value": round(wl.B * steps / (ms / 1e3), 1),
             "ms_per_call": round(ms / steps, 4), "k": K, "kp": kp, "n_buckets": nb, "exact": kp >= K,
             "roofline": rf}
@@ -459,8 +470,7 @@ def main():
     rf["kernel"] = dom
     rf["ms_per_launch"] = round(tot_ms / n_l, 4)
     rf["peak_src"] = f"{peaks['src']} ({'sustained' if rf['bound'] == 'tensor' else 'copy'})"
-    rf["traffic"] = traffic_of(args.config, dom)
-    rf["traffic_src"] = "ncu capture, profiles/k_dx2_670k.md" if rf["traffic"] else "no capture of this kernel source"
+    rf["traffic"], rf["traffic_src"] = traffic_of(args.config, dom)
     tail_ms = sum(prof[k][1] for k in prof if k.startswith("tail") or k in ("xt", "dx_reduce")) / args.steps
     tail_rf = roofline_of(work["tail"][0], work["tail"][1], tail_ms, peaks)
 

@@ -19,6 +19,7 @@
 #include "head.cu"
 #include "tail.cu"
 #include "tail_v2.cu"
+#include "dx_band.cu"
 #include "topk.cu"
 
 using namespace haste;
