@@ -230,6 +230,8 @@ cudaError_t dx_v2(const haste_plan_s& p, int B, const void* W, const void* dY, i
   v2::DxArgs a{};
   a.sh = make_args(p, B).sh;
   a.idx = p.idx_d;
+  a.dY = static_cast<const __nv_bfloat16*>(dY);
+  a.W = static_cast<const __nv_bfloat16*>(W);
   a.dX_part = part;
   a.band = t.band;
   a.n_bands = t.n_bands;

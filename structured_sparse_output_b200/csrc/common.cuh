@@ -105,6 +105,12 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* tm,
       : "memory");
 }
 
+// Hint: bring `bytes` (a multiple of 16, 16-byte aligned) of global memory into
+// L2 without waiting for them; a later load of the range then finds it there.
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
 // ---------------------------------------------------------------- cp.async
 // 16-byte global->shared copy through L2 only; src_bytes < 16 zero-fills the rest.
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {

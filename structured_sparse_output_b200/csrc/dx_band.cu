@@ -16,6 +16,8 @@ namespace v2 {
 struct DxArgs {
   TailShape sh;
   const int32_t* idx;
+  const __nv_bfloat16* dY;  // for L2 prefetches of the group-major buffer
+  const __nv_bfloat16* W;
   float* dX_part;
   int band, n_bands, n_chunks, ns;  // ns: stages of the shared-memory ring
   // element (b, g*G + j) of dY is at dY[g*dy_gstride + b*dy_rstride + j]
@@ -25,6 +27,7 @@ struct DxArgs {
 };
 
 constexpr int kMaxDxStages = 6;  // deepest ring of the dX pass
+constexpr int kDxPrefetch = 8;   // groups ahead of the ring loads that are prefetched into L2
 
 struct DxLayout {
   uint32_t dy, w, wt, rows, bars, total, dy_stride, w_stride, wt_stride;
@@ -141,9 +144,19 @@ __global__ void __launch_bounds__(kDxThreads, 1)
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       const uint32_t bytes = (uint32_t)(sh.Bp + kK) * RB;  // dY tile + weight block
+      const bool group_major = a.dy_gstride != kG;
+      // a ring load from HBM takes longer than the ring's MMA work: the tiles of
+      // later groups are requested into L2 ahead of their ring loads
+      auto prefetch = [&](int64_t g) {
+        if (group_major) prefetch_l2(a.dY + g * a.dy_gstride, (uint32_t)(sh.Bp * RB));
+        prefetch_l2(a.W + g * kG * kK, (uint32_t)(kG * kK * 2));
+        prefetch_l2(a.idx + g * kK, (uint32_t)(kK * 4));
+      };
+      for (int i = 0; i < kDxPrefetch && i < n; ++i) prefetch(g0 + i);
       int st = 0, ph = 0, issued = 0;
       for (int i = 0; i < n; ++i) {
         const int64_t g = g0 + i;
+        if (i + kDxPrefetch < n) prefetch(g + kDxPrefetch);
         if (!wait_or_abort(&empty[st], ph ^ 1, abort_flag)) break;
         ++issued;
         mbar_arrive_expect_tx(&full[st], bytes);

@@ -151,6 +151,12 @@ __global__ void __launch_bounds__(kStepThreads, 1)
     int i = half;
     for (; i < n_items; i += 2) {
       const int64_t g = gb + i;
+      // this half's next group: weight block and indices into L2 (from HBM they
+      // would stretch the gather of that group)
+      if (part == 0 && lane == 0 && i + 2 < n_items) {
+        prefetch_l2(W + (g + 2) * kG * kK, (uint32_t)(kG * kK * 2));
+        prefetch_l2(a.idx + (g + 2) * kK, (uint32_t)(kK * 4));
+      }
       // the index loads are in flight while this half waits for its stage
       int idx_cur[kRows];
 #pragma unroll
