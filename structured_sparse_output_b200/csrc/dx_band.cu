@@ -30,11 +30,10 @@ constexpr int kMaxDxStages = 6;  // deepest ring of the dX pass
 constexpr int kDxPrefetch = 8;   // groups ahead of the ring loads that are prefetched into L2
 
 struct DxLayout {
-  uint32_t dy, w, wt, rows, bars, total, dy_stride, w_stride, wt_stride;
+  uint32_t dy, w, wt, bars, total, dy_stride, w_stride, wt_stride;
 };
 // Shared memory of the dX pass: ns stages of (dY tile [Bp][G], weight block
-// [k/64][G][64], densified weight block [band][G]), the rows each slot wrote into
-// every densified block, and the barriers.
+// [k/64][G][64], densified weight block [band][G]) and the barriers.
 __host__ __device__ inline DxLayout dx_layout(int Bp, int band, int k, int G, int ns) {
   DxLayout L;
   L.dy_stride = (uint32_t)((Bp * G * 2 + 1023) & ~1023);
@@ -47,8 +46,6 @@ __host__ __device__ inline DxLayout dx_layout(int Bp, int band, int k, int G, in
   off += ns * L.w_stride;
   L.wt = off;
   off += ns * L.wt_stride;
-  L.rows = off;
-  off += ns * 128 * 4;
   L.bars = off;
   off += 512;
   L.total = off + 1024;
@@ -56,7 +53,7 @@ __host__ __device__ inline DxLayout dx_layout(int Bp, int band, int k, int G, in
 }
 
 // ========================================================== k_dx_band
-constexpr int kDxThreads = 192;  // producer warp, MMA warp, 4 densify / epilogue warps
+constexpr int kDxThreads = 320;  // producer warp, MMA warp, two sets of 4 densify / epilogue warps
 
 // The dX pass as one dense product per group and feature band.  For a band of
 // NB features [f0, f0+NB), the densified weight block Wt_g[n][j'] (n over the
@@ -70,14 +67,16 @@ constexpr int kDxThreads = 192;  // producer warp, MMA warp, 4 densify / epilogu
 // accumulators of NB columns) and a chunk of groups:
 //   producer (warp 0, one thread): the dY tile (Bp x G, K-major, swizzled rows of
 //     2G bytes) and the G x k weight block into a stage of the ring with TMA;
-//   densify (warps 2-5, the thread of slot s): clears the row it wrote into this
-//     stage's Wt block NS groups ago, then (after a barrier of the four warps)
-//     copies column s of the weight block into the Wt row of the slot's feature
-//     when it falls in the band;
+//   densify (two sets of four warps, warps 2-5 for the even groups of the chunk,
+//     6-9 for the odd ones; the thread of slot s): clears the Wt row of slot s's
+//     feature in group i - NS (the previous user of the stage, read from the
+//     index array), then, after a barrier of its set, copies column s of the
+//     weight block into the Wt row of the slot's feature when it falls in the
+//     band;
 //   MMA (warp 1): D[t] += dY_g[128t.., :] . Wt_g^T for each batch tile t;
-//   epilogue (warps 2-5): the TMEM accumulators to the chunk partial.
-// Every densify warp runs the same number of iterations (one per group of the
-// chunk), so the named barrier always matches; a wait that runs out raises the
+//   epilogue (warps 2-9): the TMEM accumulators to the chunk partial.
+// The warps of a set run the same number of iterations (one per group of the
+// set), so its named barrier always matches; a wait that runs out raises the
 // abort flag and the remaining iterations skip their work.
 template <int kG, int kK>
 __global__ void __launch_bounds__(kDxThreads, 1)
@@ -101,7 +100,6 @@ __global__ void __launch_bounds__(kDxThreads, 1)
   auto DYS = [&](int st) -> uint32_t { return base + Lo.dy + st * Lo.dy_stride; };
   auto WS = [&](int st) -> uint32_t { return base + Lo.w + st * Lo.w_stride; };
   auto WT = [&](int st) -> uint32_t { return base + Lo.wt + st * Lo.wt_stride; };
-  int* rows_used = reinterpret_cast<int*>(gbase + Lo.rows);  // [NS][128]: Wt row a slot wrote, or -1
   uint64_t* bars = reinterpret_cast<uint64_t*>(gbase + Lo.bars);
   uint64_t* full = bars;                      // [NS] dY tile + weight block landed (1 + tx bytes)
   uint64_t* empty = full + kMaxDxStages;      // [NS] both read: MMA commit + 4 densify warps
@@ -115,7 +113,7 @@ __global__ void __launch_bounds__(kDxThreads, 1)
   if (threadIdx.x == 0) {
     for (int st = 0; st < NS; ++st) {
       mbar_init(&full[st], 1);
-      mbar_init(&empty[st], 5);
+      mbar_init(&empty[st], 5);   // MMA commit + the 4 warps of one densify set
       mbar_init(&wt_full[st], 4);
       mbar_init(&wt_empty[st], 1);
     }
@@ -132,8 +130,7 @@ __global__ void __launch_bounds__(kDxThreads, 1)
     // zero Wt blocks, no rows written yet
     const int t = threadIdx.x - 64;
     uint4* wt0 = reinterpret_cast<uint4*>(gbase + Lo.wt);
-    for (uint32_t e = (uint32_t)t; e < (uint32_t)NS * Lo.wt_stride / 16; e += 128) wt0[e] = make_uint4(0, 0, 0, 0);
-    for (int e = t; e < NS * 128; e += 128) rows_used[e] = -1;
+    for (uint32_t e = (uint32_t)t; e < (uint32_t)NS * Lo.wt_stride / 16; e += 256) wt0[e] = make_uint4(0, 0, 0, 0);
   }
   tc_fence_before();
   __syncthreads();
@@ -203,40 +200,44 @@ __global__ void __launch_bounds__(kDxThreads, 1)
     __syncwarp();
   } else {
     // ----------------------------------------------- densify, then epilogue
-    const int s = threadIdx.x - 64;  // this thread's slot
+    const int set = (w - 2) >> 2;          // groups i = set, set + 2, ...
+    const int s = (threadIdx.x - 64) & 127;  // this thread's slot
     const bool slot_ok = s < kK;
     // column s of a weight block: 64-slot block s/64, 16-byte chunk (s%64)/8 of each
     // 128-byte row (TMA 128-byte swizzle), element s%8
     const uint32_t wcol = (uint32_t)((s >> 6) * kG * 128 + (s & 7) * 2);
     const uint32_t wchunk = (uint32_t)((s & 63) >> 3);
-    int fa = 0, fb = 0, fc = 0;  // the slot's feature, three groups ahead
-    if (slot_ok) {
-      if (n > 0) fa = a.idx[g0 * kK + s];
-      if (n > 1) fb = a.idx[(g0 + 1) * kK + s];
-      if (n > 2) fc = a.idx[(g0 + 2) * kK + s];
-    }
-    int st = 0, ph = 0;
-    for (int i = 0; i < n; ++i) {
-      const int f = fa - f0;
-      const bool act = slot_ok && f >= 0 && f < nf;
+    // the slot's feature in group i of the chunk (-1: no such group or slot)
+    auto feat = [&](int i) -> int { return slot_ok && i >= 0 && i < n ? a.idx[(g0 + i) * kK + s] : -1; };
+    // features of this set's next three groups, and of the groups NS before them
+    // (the previous users of the same ring stages), loaded ahead
+    int fa = feat(set), fb = feat(set + 2), fc = feat(set + 4);
+    int oa = feat(set - NS), ob = feat(set + 2 - NS), oc = feat(set + 4 - NS);
+    for (int i = set; i < n; i += 2) {
+      const int st = i % NS;
+      const uint32_t ph = (uint32_t)(i / NS) & 1u;
+      const int f = fa - f0, r = oa - f0;
+      const bool act = fa >= 0 && f >= 0 && f < nf;
+      const bool old = oa >= 0 && r >= 0 && r < nf;
       fa = fb;
       fb = fc;
-      if (slot_ok && i + 3 < n) fc = a.idx[(g0 + i + 3) * kK + s];
+      fc = feat(i + 6);
+      oa = ob;
+      ob = oc;
+      oc = feat(i + 6 - NS);
       uint8_t* wt = gbase + Lo.wt + st * Lo.wt_stride;
-      int* ru = rows_used + st * 128 + s;
       // the MMA of group i - NS has read this stage's Wt block: clear its rows
-      const bool ok = __all_sync(0xffffffffu, wait_or_abort(&wt_empty[st], ph ^ 1, abort_flag));
+      const bool ok = __all_sync(0xffffffffu, wait_or_abort(&wt_empty[st], ph ^ 1u, abort_flag));
       if (ok) {
-        const int r = *ru;
-        if (r >= 0) {
+        if (old) {
 #pragma unroll
           for (int cc = 0; cc < kG / 8; ++cc)
             *reinterpret_cast<uint4*>(wt + swz_rows((uint32_t)(r * RB + cc * 16), RB)) = make_uint4(0, 0, 0, 0);
         }
       }
       // every old row is clear before any new row is written (two slots of
-      // consecutive groups may share a feature)
-      named_bar(1, 128);
+      // different groups may share a feature)
+      named_bar(1 + set, 128);
       const bool ok2 = ok && __all_sync(0xffffffffu, wait_or_abort(&full[st], ph, abort_flag));
       if (ok2) {
         if (act) {
@@ -254,17 +255,12 @@ __global__ void __launch_bounds__(kDxThreads, 1)
             *reinterpret_cast<uint4*>(wt + swz_rows((uint32_t)(f * RB + cc * 16), RB)) =
                 make_uint4(pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
         }
-        *ru = act ? f : -1;
         fence_proxy_async_smem();
       }
       __syncwarp();
       if (lane == 0 && ok2) {
         mbar_arrive(&empty[st]);
         mbar_arrive(&wt_full[st]);
-      }
-      if (++st == NS) {
-        st = 0;
-        ph ^= 1;
       }
     }
     // ------------------------------------------------------------ epilogue
@@ -273,9 +269,10 @@ __global__ void __launch_bounds__(kDxThreads, 1)
     const int q = w & 3;  // TMEM lane quarter: batch rows 32q.. of each tile
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     if (fin) {
-      for (int t = 0; t < MT; ++t) {
+      // two batch tiles: one per set; one tile: the sets take alternate 16-column chunks
+      for (int t = MT == 2 ? set : 0; t < (MT == 2 ? set + 1 : 1); ++t) {
         const int b = t * 128 + q * 32 + lane;
-        for (int c0 = 0; c0 < NB; c0 += 16) {
+        for (int c0 = MT == 2 ? 0 : 16 * set; c0 < NB; c0 += MT == 2 ? 16 : 32) {
           float v[16];
           tmem_ld16(tmem + lane_off + (uint32_t)(t * 256 + c0), v);
           tmem_wait_ld();
