@@ -678,13 +678,10 @@ haste_status_t haste_bce_step(haste_plan_t p, int32_t B, haste_dtype_t dt, const
       e = dt == HASTE_BF16 ? tail::launch_backward_dx<__nv_bfloat16>(a, true, s)
                            : tail::launch_backward_dx<float>(a, true, s);
   }
-  if (e == cudaSuccess) {
+  if (e == cudaSuccess) {  // the chunk partials of dX and, with a loss pointer, the loss partials
     ProfScope ps("dx_reduce", s);
-    e = tail::launch_dx_reduce(a.dX_part, dX, t.n_chunks, p->d, Bp, B, accumulate, s);
-  }
-  if (e == cudaSuccess && loss) {
-    ProfScope ps("loss_reduce", s);
-    e = tail::launch_loss_reduce(a.loss_part, grid, grad_scale, loss, s);
+    e = tail::launch_dx_reduce(a.dX_part, dX, t.n_chunks, p->d, Bp, B, accumulate, s, loss ? a.loss_part : nullptr,
+                               grid, grad_scale, loss);
   }
   return e == cudaSuccess ? HASTE_OK : cuda_fail(e, "haste_bce_step launch");
 }

@@ -213,9 +213,10 @@ __global__ void __launch_bounds__(kDxThreads, 1)
     // (the previous users of the same ring stages), loaded ahead
     int fa = feat(set), fb = feat(set + 2), fc = feat(set + 4);
     int oa = feat(set - NS), ob = feat(set + 2 - NS), oc = feat(set + 4 - NS);
+    // ring position of group i, advanced by two groups per iteration (NS >= 2)
+    int st = set;
+    uint32_t ph = 0;
     for (int i = set; i < n; i += 2) {
-      const int st = i % NS;
-      const uint32_t ph = (uint32_t)(i / NS) & 1u;
       const int f = fa - f0, r = oa - f0;
       const bool act = fa >= 0 && f >= 0 && f < nf;
       const bool old = oa >= 0 && r >= 0 && r < nf;
@@ -261,6 +262,10 @@ __global__ void __launch_bounds__(kDxThreads, 1)
       if (lane == 0 && ok2) {
         mbar_arrive(&empty[st]);
         mbar_arrive(&wt_full[st]);
+      }
+      if ((st += 2) >= NS) {
+        st -= NS;
+        ph ^= 1u;
       }
     }
     // ------------------------------------------------------------ epilogue

@@ -448,26 +448,53 @@ __global__ void __launch_bounds__(kThreads, 1) k_backward_dx(TailArgs a) {
   tmem_teardown(tmem, ncols);
 }
 
-// dX[b, f] (+)= sum over chunks c ascending of dX_part[c, f, b].
+// One warp: *loss = scale * sum of part[0..n) in fp64, in a fixed order (lane j
+// adds part[j], part[j+32], ... in turn, then a butterfly over the lanes), so
+// the result is the same on every run.
+__device__ __forceinline__ void loss_sum(const float* __restrict__ part, int n, float scale, float* loss) {
+  double t = 0.0;
+  for (int i = (int)(threadIdx.x & 31); i < n; i += 32) t += (double)part[i];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+  if ((threadIdx.x & 31) == 0) *loss = (float)(t * (double)scale);
+}
+
+// dX[b, f] (+)= sum over chunks c ascending of dX_part[c, f, b].  With
+// loss_part, the first warp of block (0, 0) also writes the loss, as
+// k_loss_reduce does.
 __global__ void __launch_bounds__(256) k_dx_reduce(const float* __restrict__ P, float* __restrict__ dX, int C,
-                                                   int d, int Bp, int B, int accumulate) {
+                                                   int d, int Bp, int B, int accumulate,
+                                                   const float* __restrict__ loss_part, int n_loss, float scale,
+                                                   float* __restrict__ loss) {
   __shared__ float tile[32][33];
   const int f0 = blockIdx.x * 32, b0 = blockIdx.y * 32;
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
-  for (int i = ty; i < 32; i += 8) {
-    const int f = f0 + i, bb = b0 + tx;
-    float s = 0.f;
-    if (f < d)
-      for (int c = 0; c < C; ++c) s += P[((int64_t)c * d + f) * Bp + bb];
-    tile[i][tx] = s;
+  if (loss_part && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x < 32) loss_sum(loss_part, n_loss, scale, loss);
+  // four feature rows per thread, summed side by side so that their loads are in
+  // flight together; every element still adds its chunks in ascending order
+  const int64_t cs = (int64_t)d * Bp;
+  const float* p = P + (int64_t)(f0 + ty) * Bp + b0 + tx;
+  const bool k0 = f0 + ty < d, k1 = f0 + ty + 8 < d, k2 = f0 + ty + 16 < d, k3 = f0 + ty + 24 < d;
+  float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+#pragma unroll 4
+  for (int c = 0; c < C; ++c) {
+    const float* q = p + c * cs;
+    if (k0) s0 += q[0];
+    if (k1) s1 += q[8 * Bp];
+    if (k2) s2 += q[16 * Bp];
+    if (k3) s3 += q[24 * Bp];
   }
+  tile[ty][tx] = s0;
+  tile[ty + 8][tx] = s1;
+  tile[ty + 16][tx] = s2;
+  tile[ty + 24][tx] = s3;
   __syncthreads();
   for (int i = ty; i < 32; i += 8) {
     const int bb = b0 + i, f = f0 + tx;
     if (bb < B && f < d) {
       const float v = tile[tx][i];
-      float* p = dX + (int64_t)bb * d + f;
-      *p = accumulate ? *p + v : v;
+      float* q = dX + (int64_t)bb * d + f;
+      *q = accumulate ? *q + v : v;
     }
   }
 }
@@ -619,11 +646,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_step(TailArgs a) {
 
 // loss = scale * sum of the per-CTA partials in ascending CTA order (double).
 __global__ void k_loss_reduce(const float* __restrict__ part, int n, float scale, float* loss) {
-  if (threadIdx.x == 0 && blockIdx.x == 0) {
-    double s = 0.0;
-    for (int i = 0; i < n; ++i) s += (double)part[i];
-    *loss = (float)(s * (double)scale);
-  }
+  if (blockIdx.x == 0 && threadIdx.x < 32) loss_sum(part, n, scale, loss);
 }
 
 // Self-test of the bounded-wait path: one thread waits on an mbarrier that no one
@@ -715,9 +738,10 @@ cudaError_t launch_backward_dx(const TailArgs& a, bool from_step, cudaStream_t s
 }
 
 cudaError_t launch_dx_reduce(const float* P, float* dX, int C, int d, int Bp, int B, int accumulate,
-                             cudaStream_t st) {
+                             cudaStream_t st, const float* loss_part = nullptr, int n_loss = 0,
+                             float scale = 0.f, float* loss = nullptr) {
   dim3 grid((d + 31) / 32, Bp / 32);
-  k_dx_reduce<<<grid, 256, 0, st>>>(P, dX, C, d, Bp, B, accumulate);
+  k_dx_reduce<<<grid, 256, 0, st>>>(P, dX, C, d, Bp, B, accumulate, loss_part, n_loss, scale, loss);
   return cudaGetLastError();
 }
 
