@@ -81,7 +81,11 @@ def algorithmic(wl):
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) of a
 # kernel from one ncu capture (summaries under profiles/), valid only for the
 # source file it was taken on: (config, timed region) -> (bytes, source digest).
-TRAFFIC = {}
+TRAFFIC = {
+    ("670k", "tail_step"): (643.1e6, "6c87e65aba6e9fd4"),
+    ("670k", "tail_dx"): (531.9e6, "2d77d886196a1fa8"),
+    ("670k", "topk_score"): (186.2e6, "a08fbb472ccd8c70"),
+}
 # timed region -> (source file under csrc/, kernel name in the ncu summaries)
 KERNELS = {"tail_step": ("tail_v2.cu", "k_step2"), "tail_dx": ("dx_band.cu", "k_dx_band"),
            "topk_score": ("topk.cu", "k_topk")}
