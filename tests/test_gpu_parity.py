@@ -54,6 +54,12 @@ TAIL_CASES = [
     dict(B=512, d=1024, n_groups=256, G=16, k=128, dtype="bf16"),
     dict(B=128, d=512, n_groups=64, G=128, k=64, dtype="bf16"),
     dict(B=64, d=96, n_groups=40, G=48, k=64, dtype="bf16"),
+    # dX band kernel: one 128-row batch tile, G = 16 (32-byte rows), one band of 208 cut to 200 features
+    dict(B=100, d=200, n_groups=150, G=16, k=64, dtype="bf16"),
+    # fewer groups than group chunks: one group per CTA, one batch tile
+    dict(B=64, d=768, n_groups=5, G=32, k=128, dtype="bf16"),
+    # four bands, the last one 232 features wide
+    dict(B=256, d=1000, n_groups=97, G=16, k=128, dtype="bf16"),
 ]
 
 
@@ -110,6 +116,7 @@ STEP_CASES = [
     dict(B=256, d=768, n_groups=300, G=64, k=128, dtype="bf16", H=128, p=8),
     dict(B=32, d=256, n_groups=256, G=16, k=32, dtype="f32", H=32, p=5),
     dict(B=300, d=512, n_groups=200, G=16, k=64, dtype="bf16", H=0, p=6),
+    dict(B=100, d=256, n_groups=120, G=16, k=64, dtype="bf16", H=0, p=5),   # one batch tile, G = 16
 ]
 
 
