@@ -4,9 +4,10 @@
 //
 // k_dx_band -- per CTA (feature band, group chunk), every batch row: warp 0 loads
 //   each group's dY tile and G x k weight block into a shared-memory ring with
-//   TMA, warps 2-5 densify the weight block over the band, warp 1 issues one MMA
-//   per 128-row batch tile into TMEM accumulators, and warps 2-5 write the chunk
-//   partial at the end.  k_dx_reduce (tail.cu) sums the chunk partials in order.
+//   TMA, warps 2-9 (two sets of four, alternate groups) densify the weight block
+//   over the band, warp 1 issues one MMA per 128-row batch tile into TMEM
+//   accumulators, and warps 2-9 write the chunk partial at the end.  k_dx_reduce
+//   (tail.cu) sums the chunk partials in order.
 
 #include "tail.cuh"
 
