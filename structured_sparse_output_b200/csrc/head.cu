@@ -238,10 +238,11 @@ cudaError_t run_gemm(const GemmArgs& a, int splits, cudaStream_t st) {
 
 namespace head {
 
-// Work split of dXh (K = H can be long): K chunks of a multiple of the stage depth.
+// Work split of dXh (K = H can be long): K chunks of a multiple of the stage depth,
+// about 512 long, so that the few output tiles (B/128 x d/128) still fill the SMs.
 int dxh_splits(int H, int elem) {
   const int BK = 2 * (128 / elem);
-  int s = H / 1024;
+  int s = H / 512;
   if (s < 1) s = 1;
   if (s > 32) s = 32;
   while (s > 1 && ((H + s - 1) / s) % BK) --s;
