@@ -15,7 +15,8 @@ namespace haste {
 namespace {
 
 constexpr int kGThreads = 128;
-constexpr int kBM = 128, kBN = 128;
+constexpr int kBM = 128;
+constexpr int kFwdN = 64;  // output tile width of the forward (B x H has few 128-wide tiles)
 
 enum Epi : int { kEpiStore = 0, kEpiStoreF32 = 1, kEpiPartial = 2, kEpiBce = 3 };
 
@@ -34,20 +35,22 @@ struct GemmArgs {
   float* loss_part;
 };
 
-// Stage a 128 x BK tile of an operand whose rows are the M (or N) index.
-template <typename T, bool kMN>
+// Stage a kRows x BK tile of an operand whose rows are the M (or N) index
+// (kRows = 128, or 64 for a K-major operand).
+template <typename T, bool kMN, int kRows = 128>
 __device__ __forceinline__ void load_operand(uint32_t s, const T* __restrict__ p, int64_t ld, int rows, int K,
                                              int r0, int k0, int BK) {
   constexpr int CW = 16 / sizeof(T);
+  static_assert(kRows == 128 || (kRows == 64 && !kMN), "64-row tiles are K-major only");
   if constexpr (!kMN) {
     // K-major: [k-block][row][128B]
     const int cpr = BK / CW;
-    for (int i = threadIdx.x; i < 128 * cpr; i += blockDim.x) {
+    for (int i = threadIdx.x; i < kRows * cpr; i += blockDim.x) {
       const int r = i / cpr, cc = i % cpr;
       const int gr = r0 + r, gk = k0 + cc * CW;
       const bool in = gr < rows && gk < K;
       const T* src = in ? p + (int64_t)gr * ld + gk : p;
-      const uint32_t off = (uint32_t)((cc >> 3) * 128 * 128 + r * 128 + (cc & 7) * 16);
+      const uint32_t off = (uint32_t)((cc >> 3) * kRows * 128 + r * 128 + (cc & 7) * 16);
       cp_async16(s + sw128(off), src, in ? 16u : 0u);
     }
   } else {
@@ -64,17 +67,18 @@ __device__ __forceinline__ void load_operand(uint32_t s, const T* __restrict__ p
   }
 }
 
-template <typename T, bool kMN>
+template <typename T, bool kMN, int kRows = 128>
 __device__ __forceinline__ uint64_t operand_desc(uint32_t s, int kk, int BK) {
   constexpr int R = 128 / sizeof(T), KI = Elem<T>::kMmaK;
   if constexpr (!kMN) {
-    return make_sdesc(s + (uint32_t)(((kk * KI) / R) * 128 * 128 + (kk % (R / KI)) * 32), 16, 1024, kLayoutSw128);
+    return make_sdesc(s + (uint32_t)(((kk * KI) / R) * kRows * 128 + (kk % (R / KI)) * 32), 16, 1024,
+                      kLayoutSw128);
   } else {
     return mn_desc<T>(s + (uint32_t)(kk * KI * 128), (uint32_t)BK * 128);
   }
 }
 
-template <typename T, bool kAMN, bool kBMN, int kEpi>
+template <typename T, bool kAMN, bool kBMN, int kEpi, int kBN>
 __global__ void __launch_bounds__(kGThreads, 1) k_gemm(GemmArgs a) {
   extern __shared__ __align__(1024) uint8_t smem[];
   constexpr int R = 128 / sizeof(T), KI = Elem<T>::kMmaK;
@@ -113,7 +117,7 @@ __global__ void __launch_bounds__(kGThreads, 1) k_gemm(GemmArgs a) {
 
   for (int k0 = k_begin; k0 < k_end; k0 += BK) {
     load_operand<T, kAMN>(sa, A, a.lda, a.M, k_end, m0, k0, BK);
-    load_operand<T, kBMN>(sb, Bm, a.ldb, a.N, k_end, n0, k0, BK);
+    load_operand<T, kBMN, kBN>(sb, Bm, a.ldb, a.N, k_end, n0, k0, BK);
     cp_async_commit();
     cp_async_wait_all();
     fence_proxy_async_smem();
@@ -121,7 +125,7 @@ __global__ void __launch_bounds__(kGThreads, 1) k_gemm(GemmArgs a) {
     if (threadIdx.x == 0) {
       tc_fence_after();
       for (int kk = 0; kk < BK / KI; ++kk)
-        mma_ss<Elem<T>::kTF32>(tmem, operand_desc<T, kAMN>(sa, kk, BK), operand_desc<T, kBMN>(sb, kk, BK), idesc,
+        mma_ss<Elem<T>::kTF32>(tmem, operand_desc<T, kAMN>(sa, kk, BK), operand_desc<T, kBMN, kBN>(sb, kk, BK), idesc,
                                (k0 > k_begin || kk > 0) ? 1u : 0u);
       mma_commit(bar);
     }
@@ -146,7 +150,7 @@ __global__ void __launch_bounds__(kGThreads, 1) k_gemm(GemmArgs a) {
         for (int p = a.pos_ptr[m]; p < a.pos_ptr[m + 1]; ++p) {
           const int l = a.pos_ids[p] - n0;
           if (l >= 0 && l < 64) ym0 |= 1ull << l;
-          else if (l >= 64 && l < 128) ym1 |= 1ull << (l - 64);
+          else if (l >= 64 && l < kBN) ym1 |= 1ull << (l - 64);
         }
     }
     for (int c = 0; c < kBN; c += 16) {
@@ -222,11 +226,11 @@ __global__ void k_split_reduce(const float* __restrict__ P, float* __restrict__ 
   }
 }
 
-template <typename T, bool kAMN, bool kBMN, int kEpi>
+template <typename T, bool kAMN, bool kBMN, int kEpi, int kBN = 128>
 cudaError_t run_gemm(const GemmArgs& a, int splits, cudaStream_t st) {
   constexpr int BK = 2 * (128 / (int)sizeof(T));
   const size_t smem = 1024 + (size_t)(kBM + kBN) * BK * sizeof(T) + 64;
-  auto kern = k_gemm<T, kAMN, kBMN, kEpi>;
+  auto kern = k_gemm<T, kAMN, kBMN, kEpi, kBN>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((a.M + kBM - 1) / kBM, (a.N + kBN - 1) / kBN, splits);
@@ -249,7 +253,7 @@ int dxh_splits(int H, int elem) {
   return s;
 }
 
-int fwd_tiles(int B, int H) { return ((B + kBM - 1) / kBM) * ((H + kBN - 1) / kBN); }
+int fwd_tiles(int B, int H) { return ((B + kBM - 1) / kBM) * ((H + kFwdN - 1) / kFwdN); }
 
 template <typename T>
 cudaError_t forward(int B, int H, int d, const void* Xh, const void* Wh, void* out, const int32_t* pos_ptr,
@@ -270,9 +274,9 @@ cudaError_t forward(int B, int H, int d, const void* Xh, const void* Wh, void* o
     a.pos_ids = pos_ids;
     a.scale = scale;
     a.loss_part = loss_part;
-    return run_gemm<T, false, false, kEpiBce>(a, 1, st);
+    return run_gemm<T, false, false, kEpiBce, kFwdN>(a, 1, st);
   }
-  return run_gemm<T, false, false, kEpiStore>(a, 1, st);
+  return run_gemm<T, false, false, kEpiStore, kFwdN>(a, 1, st);
 }
 
 // dWh = dY_h^T . Xh : A(m=h, k=b) = dY_h[b, h] (MN-major), B(n=f, k=b) = Xh[b, f] (MN-major)
