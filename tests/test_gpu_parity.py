@@ -60,6 +60,9 @@ TAIL_CASES = [
     dict(B=64, d=768, n_groups=5, G=32, k=128, dtype="bf16"),
     # four bands, the last one 232 features wide
     dict(B=256, d=1000, n_groups=97, G=16, k=128, dtype="bf16"),
+    # degenerate counts: a batch of one row; a single group (one chunk, one CTA per band)
+    dict(B=1, d=256, n_groups=50, G=32, k=64, dtype="bf16"),
+    dict(B=37, d=256, n_groups=1, G=32, k=64, dtype="bf16"),
 ]
 
 
@@ -117,6 +120,8 @@ STEP_CASES = [
     dict(B=32, d=256, n_groups=256, G=16, k=32, dtype="f32", H=32, p=5),
     dict(B=300, d=512, n_groups=200, G=16, k=64, dtype="bf16", H=0, p=6),
     dict(B=100, d=256, n_groups=120, G=16, k=64, dtype="bf16", H=0, p=5),   # one batch tile, G = 16
+    dict(B=1, d=256, n_groups=40, G=32, k=64, dtype="bf16", H=16, p=3),     # a batch of one row
+    dict(B=37, d=256, n_groups=1, G=32, k=64, dtype="bf16", H=0, p=2),      # a single group
 ]
 
 
