@@ -6,11 +6,13 @@
 //   warps 0-3  producers: the gather-once tile X[:, I_g] (k rows of X^T) and the
 //              G x k weight block, staged with cp.async into a 2-stage ring; warps
 //              0 and 2 fill stage 0, warps 1 and 3 stage 1;
-//   warp 4     MMA issuer (one thread): forward of group i+1 is issued before the
-//              dW of group i, so the tensor core works while the epilogue runs;
+//   warp 4     MMA issuer (one thread): issues each group's forward and dW
+//              product as soon as its inputs are ready, so the tensor core works
+//              while the epilogue runs;
 //   warps 5-12 epilogue: logits leave TMEM only as the BCE gradient (bf16, to
 //              shared memory for the dW product and to the group-major gradient
-//              buffer of the dX pass), then dW is read out of TMEM.
+//              buffer of the dX pass); the BCE of group i+1 comes before the dW
+//              readout of group i, so the dW product runs behind it.
 //
 // The dX pass that reads the gradient buffer is in dx_band.cu.
 
@@ -188,45 +190,78 @@ __global__ void __launch_bounds__(kStepThreads, 1)
     cp_async_wait_all();
   } else if (w == kStepMma) {
     // ------------------------------------------------------------ MMA issuer
+    // Forwards and dW products are issued as their inputs become ready, not in a
+    // fixed interleave: fwd(j) needs its gathered stage (full) and F(j&1) free,
+    // which holds once dW(j-2) was issued (its BCE had finished reading F);
+    // dW(j) needs the BCE of j (dy_full) and D(j&1) read out for j-2
+    // (tmem_empty).  Lane 0 polls; the decisions are broadcast so the warp stays
+    // converged.  No progress for kWaitLimitNs raises the abort flag.
     const uint32_t idesc_f = make_idesc(1, 1, 0, 128, kG);
     const uint32_t idesc_w = make_idesc(1, 0, 1, 128, kG);
-    auto issue_fwd = [&](int i) -> bool {
-      const int s = i & 1;
-      if (!wait_or_abort(&tmem_empty[s], ((i >> 1) & 1) ^ 1, abort_flag)) return false;
-      if (!wait_or_abort(&full[s], (i >> 1) & 1, abort_flag)) return false;
-      tc_fence_after();
-      if (lane == 0) {
-        for (int t = 0; t < n_bt; ++t)
-          for (int kk = 0; kk < kK / 16; ++kk) {
-            const uint64_t ad = make_sdesc(XG(s) + (uint32_t)(t * 2 * kK * 128 + kk * 16 * 128), (uint32_t)kK * 128,
-                                           1024, kLayoutSw128);
-            const uint64_t bd =
-                make_sdesc(WG(s) + (uint32_t)((kk / 4) * kG * 128 + (kk % 4) * 32), 16, 1024, kLayoutSw128);
-            mma_ss<false>(F(s) + (uint32_t)(t * kG), ad, bd, idesc_f, kk > 0 ? 1u : 0u);
+    int nf = 0, nd = 0;
+    uint64_t t_last = globaltimer_ns();
+    while (nd < n_items) {
+      if (*abort_flag) break;
+      bool did = false;
+      if (nf < n_items && nf <= nd + 1) {
+        const int s = nf & 1;
+        const bool rdy = __shfl_sync(0xffffffffu, lane == 0 ? mbar_try_wait(&full[s], (nf >> 1) & 1) : false, 0);
+        if (rdy) {
+          if (lane == 0) {
+            tc_fence_after();
+            for (int t = 0; t < n_bt; ++t)
+              for (int kk = 0; kk < kK / 16; ++kk) {
+                const uint64_t ad = make_sdesc(XG(s) + (uint32_t)(t * 2 * kK * 128 + kk * 16 * 128),
+                                               (uint32_t)kK * 128, 1024, kLayoutSw128);
+                const uint64_t bd =
+                    make_sdesc(WG(s) + (uint32_t)((kk / 4) * kG * 128 + (kk % 4) * 32), 16, 1024, kLayoutSw128);
+                mma_ss<false>(F(s) + (uint32_t)(t * kG), ad, bd, idesc_f, kk > 0 ? 1u : 0u);
+              }
+            mma_commit(&fwd_full[s]);
           }
-        mma_commit(&fwd_full[s]);
-      }
-      __syncwarp();
-      return true;
-    };
-    bool ok = n_items > 0 ? issue_fwd(0) : true;
-    for (int i = 0; ok && i < n_items; ++i) {
-      if (i + 1 < n_items && !issue_fwd(i + 1)) break;
-      const int s = i & 1;
-      if (!wait_or_abort(&dy_full[s], (i >> 1) & 1, abort_flag)) break;
-      tc_fence_after();
-      if (lane == 0) {
-        for (int kk = 0; kk < Bp / 16; ++kk) {
-          const int b = kk * 16;
-          const uint64_t ad =
-              make_sdesc(XG(s) + (uint32_t)((b / 64) * kK * 128 + (kk % 4) * 32), 16, 1024, kLayoutSw128);
-          const uint64_t bd = make_sdesc(base + DY(s) + (uint32_t)(b * RB), 16, 8 * RB, layout_for_rows(RB));
-          mma_ss<false>(D(s), ad, bd, idesc_w, kk > 0 ? 1u : 0u);
+          __syncwarp();
+          ++nf;
+          did = true;
         }
-        mma_commit(&dw_full[s]);
-        mma_commit(&empty[s]);
       }
-      __syncwarp();
+      if (nd < nf) {
+        const int s = nd & 1;
+        const bool rdy = __shfl_sync(0xffffffffu,
+                                     lane == 0 ? (mbar_try_wait(&dy_full[s], (nd >> 1) & 1) &&
+                                                  mbar_try_wait(&tmem_empty[s], ((nd >> 1) & 1) ^ 1))
+                                               : false,
+                                     0);
+        if (rdy) {
+          if (lane == 0) {
+            tc_fence_after();
+            for (int kk = 0; kk < Bp / 16; ++kk) {
+              const int b = kk * 16;
+              const uint64_t ad =
+                  make_sdesc(XG(s) + (uint32_t)((b / 64) * kK * 128 + (kk % 4) * 32), 16, 1024, kLayoutSw128);
+              const uint64_t bd = make_sdesc(base + DY(s) + (uint32_t)(b * RB), 16, 8 * RB, layout_for_rows(RB));
+              mma_ss<false>(D(s), ad, bd, idesc_w, kk > 0 ? 1u : 0u);
+            }
+            mma_commit(&dw_full[s]);
+            mma_commit(&empty[s]);
+          }
+          __syncwarp();
+          ++nd;
+          did = true;
+        }
+      }
+      if (did) {
+        t_last = globaltimer_ns();
+      } else {
+        if (globaltimer_ns() - t_last > kWaitLimitNs) {
+          if (lane == 0) {
+            *abort_flag = 1;
+            record_error(kErrTimeout);
+          }
+          __syncwarp();
+          break;
+        }
+        __nanosleep(32);
+      }
     }
   } else {
     // ------------------------------------------------------------- epilogue
@@ -249,10 +284,10 @@ __global__ void __launch_bounds__(kStepThreads, 1)
 #pragma unroll
       for (int e = 0; e < kMaxPosReg; ++e) pos[t][e] = e < npos[t] ? a.pos_ids[pbeg[t] + e] : -1;
     }
-    for (int i = 0; i < n_items; ++i) {
+    auto bce = [&](int i) -> bool {
       const int64_t g = gb + i;
       const int s = i & 1;
-      if (!wait_or_abort(&fwd_full[s], (i >> 1) & 1, abort_flag)) break;
+      if (!wait_or_abort(&fwd_full[s], (i >> 1) & 1, abort_flag)) return false;
       tc_fence_after();
       const int64_t l0 = g * kG + hh * CH;  // first label of this warp's columns
       uint8_t* dyrow = gbase + DY(s);
@@ -318,7 +353,12 @@ __global__ void __launch_bounds__(kStepThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&dy_full[s]);
-      if (!wait_or_abort(&dw_full[s], (i >> 1) & 1, abort_flag)) break;
+      return true;
+    };
+    auto readout = [&](int i) -> bool {
+      const int64_t g = gb + i;
+      const int s = i & 1;
+      if (!wait_or_abort(&dw_full[s], (i >> 1) & 1, abort_flag)) return false;
       tc_fence_after();
       // dW readout: row = slot r, columns = this warp's labels
 #pragma unroll
@@ -337,6 +377,12 @@ __global__ void __launch_bounds__(kStepThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tmem_empty[s]);
+      return true;
+    };
+    bool ok = n_items > 0 ? bce(0) : true;
+    for (int i = 0; ok && i < n_items; ++i) {
+      if (i + 1 < n_items && !bce(i + 1)) break;
+      if (!readout(i)) break;
     }
     // deterministic loss reduction over the 8 epilogue warps (named barrier 1)
     float v = loss_acc;
