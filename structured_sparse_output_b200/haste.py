@@ -103,6 +103,8 @@ def _np_ptr(a: np.ndarray):
 def _tptr(t) -> Optional[int]:
     if t is None:
         return None
+    if not t.is_cuda:
+        raise ValueError("tensors must be CUDA tensors (the library reads them on the GPU)")
     if not t.is_contiguous():
         raise ValueError("tensors must be contiguous")
     return t.data_ptr()

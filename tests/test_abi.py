@@ -68,3 +68,11 @@ def test_calls_fail_cleanly_without_gpu():
     st = H.lib().haste_head_forward(256, 256, 256, H.HASTE_BF16, None, None, None, None, 1.0, None, None, 0, None)
     assert st == H.HASTE_ERR_CUDA
     assert H.lib().haste_last_error()
+
+
+def test_binding_rejects_host_tensors():
+    """A host tensor's pointer never reaches a kernel: the binding refuses it."""
+    torch = pytest.importorskip("torch")
+    with pytest.raises(ValueError, match="CUDA tensors"):
+        H._tptr(torch.zeros(8))
+    assert H._tptr(None) is None
