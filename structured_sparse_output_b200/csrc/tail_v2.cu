@@ -32,8 +32,6 @@ struct StepArgs {
   float grad_scale;
 };
 
-
-
 // ------------------------------------------------------------ smem layouts
 struct StepLayout {
   uint32_t xg[2], wg[2], dy[2], bars, total;
@@ -98,7 +96,7 @@ __global__ void __launch_bounds__(kStepThreads, 1)
   uint64_t* fwd_full = bars + 4;     // [2] logits in TMEM
   uint64_t* dy_full = bars + 6;      // [2] dY in shared memory
   uint64_t* dw_full = bars + 8;      // [2] dW in TMEM
-  uint64_t* tmem_empty = bars + 10;  // [2] TMEM buffer read out
+  uint64_t* tmem_empty = bars + 10;  // [2] dW accumulator D read out
   uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 12);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
   float* red = reinterpret_cast<float*>(tslot + 2);  // 8 warp partials
