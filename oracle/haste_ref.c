@@ -297,3 +297,45 @@ void ref_topk(int dt, const void* X, const void* W, const int32_t* idx, int32_t 
     free(ci);
   }
 }
+
+/* ---- the tail loss alone, for full-size checks ------------------------------
+ * loss = scale * sum_{b,l} ( max(z,0) - z*y + log1p(exp(-|z|)) ) with
+ * z[b, l] = logits of the forward above, computed group by group without storing
+ * the B x L logits: per group, the gathered inputs X[b, idx[g, s]] and the G
+ * weight rows are widened once, then every logit is the sum over s ascending.
+ * Per-group partial sums are added in group order (the result does not depend on
+ * the thread count). */
+double ref_bce_loss(int dt, const void* X, const void* W, const int32_t* idx, int32_t B, int32_t d,
+                    int64_t n_groups, int32_t G, int32_t k, const int32_t* row_ptr, const int32_t* ids,
+                    double scale) {
+  double* part = (double*)calloc((size_t)n_groups, sizeof(double));
+  if (!part) return NAN;
+#pragma omp parallel
+  {
+    double* xg = (double*)malloc(sizeof(double) * (size_t)B * k);
+    double* wg = (double*)malloc(sizeof(double) * (size_t)G * k);
+#pragma omp for schedule(static)
+    for (int64_t g = 0; g < n_groups; ++g) {
+      for (int32_t b = 0; b < B; ++b)
+        for (int32_t s = 0; s < k; ++s) xg[(int64_t)b * k + s] = ld(X, (int64_t)b * d + idx[g * k + s], dt);
+      for (int32_t j = 0; j < G; ++j)
+        for (int32_t s = 0; s < k; ++s) wg[(int64_t)j * k + s] = ld(W, (g * G + j) * k + s, dt);
+      double acc = 0.0;
+      for (int32_t b = 0; b < B; ++b)
+        for (int32_t j = 0; j < G; ++j) {
+          const int64_t l = g * G + j;
+          double z = 0.0;
+          for (int32_t s = 0; s < k; ++s) z += xg[(int64_t)b * k + s] * wg[(int64_t)j * k + s];
+          const double y = is_positive(ids, row_ptr[b], row_ptr[b + 1], l) ? 1.0 : 0.0;
+          acc += (z > 0 ? z : 0.0) - z * y + log1p(exp(-fabs(z)));
+        }
+      part[g] = acc;
+    }
+    free(xg);
+    free(wg);
+  }
+  double loss = 0.0;
+  for (int64_t g = 0; g < n_groups; ++g) loss += part[g];
+  free(part);
+  return scale * loss;
+}

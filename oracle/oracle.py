@@ -63,6 +63,8 @@ def _load():
         lib.ref_dx_at.argtypes = [ctypes.c_int, P, P, P, P, I32, I32, I64, I32, I32, ctypes.c_int,
                                   P, P, D, I64, P, P, P]
         lib.ref_topk.argtypes = [ctypes.c_int, P, P, P, I32, I64, I32, I32, I32, I32, I32, I64, P, P, P]
+        lib.ref_bce_loss.argtypes = [ctypes.c_int, P, P, P, I32, I32, I64, I32, I32, P, P, D]
+        lib.ref_bce_loss.restype = D
         _lib = lib
     return _lib
 
@@ -162,6 +164,19 @@ def bce_step(X, W, idx, G: int, row_ptr, ids, scale: float):
     dW = backward_dw(X, dY, idx, G)
     dX = backward_dx(W, dY, idx, G, d)
     return loss, dY, dW, dX
+
+
+def bce_loss(X, W, idx, G: int, row_ptr, ids, scale: float) -> float:
+    """The fused step's tail loss alone (forward + BCE sum, no B x L logits kept),
+    for full-size checks.  X and W share one dtype."""
+    X, W, idx = _c(X), _c(W), _c(idx, np.int32)
+    if _dt(X) != _dt(W):
+        raise TypeError("bce_loss takes X and W of one dtype")
+    row_ptr, ids = _c(row_ptr, np.int32), _c(ids, np.int32)
+    B, d = X.shape
+    n_groups, k = idx.shape
+    return float(_load().ref_bce_loss(_dt(X), _ptr(X), _ptr(W), _ptr(idx), B, d, n_groups, G, k,
+                                      _ptr(row_ptr), _ptr(ids), scale))
 
 
 # ------------------------------------------------ sampled single-output checks

@@ -288,6 +288,29 @@ def test_sampled_evaluations_match_full():
                                dXf[bs, fs], rtol=1e-12, atol=1e-14)
 
 
+def test_bce_loss_alone_matches_the_pinned_step_and_closed_forms():
+    """The loss-only evaluation (no B x L logits kept) against numpy logaddexp of a
+    numpy masked-dense forward, for f32 and bf16 inputs; W = 0 gives n * ln 2."""
+    B, d, n_groups, G, k = 7, 48, 9, 4, 8
+    for dt in ("f32", "bf16"):
+        idx = I.make_idx(n_groups, k, d, 6)
+        X = I.make_normal((B, d), 1.0, 6, 1, dt)
+        W = I.make_normal((n_groups * G, k), 0.7, 6, 2, dt)
+        rp, ids = I.make_zipf_positives(B, n_groups * G, 3, 1.0, 6)
+        z = O.to_f64(X) @ _dense_w(O.to_f64(W), idx, G, d).T
+        y = np.zeros_like(z)
+        for b in range(B):
+            y[b, ids[rp[b]:rp[b + 1]]] = 1.0
+        ref = float(np.sum(np.logaddexp(0.0, z) - z * y)) / B
+        assert math.isclose(O.bce_loss(X, W, idx, G, rp, ids, 1.0 / B), ref, rel_tol=1e-12)
+        assert math.isclose(O.bce_loss(X, W, idx, G, rp, ids, 1.0 / B),
+                            O.bce_step(X, W, idx, G, rp, ids, 1.0 / B)[0], rel_tol=1e-13)
+    W0 = np.zeros((n_groups * G, k), dtype=np.float32)
+    X = I.make_normal((B, d), 1.0, 6, 1, "f32")
+    got = O.bce_loss(X, W0, I.make_idx(n_groups, k, d, 6), G, rp, ids, 0.5)
+    assert math.isclose(got, 0.5 * B * n_groups * G * math.log(2.0), rel_tol=1e-14)
+
+
 # ------------------------------------------------------------------- head
 def test_head_is_the_dense_special_case_of_the_sparse_layer():
     """A dense head over H labels is one group of G = H labels with k = d."""
@@ -417,3 +440,38 @@ def test_topk_recall_grows_with_kp_and_survivors_are_true_scores():
         assert recall >= prev
         prev = recall
     assert prev == 1.0
+
+
+def test_topk_bucket_partition_planted_logits():
+    """Buckets that do not divide the groups evenly, and K' < K.  97 groups in 13
+    buckets: bucket j = groups [floor(97 j / 13), floor(97 (j+1) / 13)), boundaries
+    0 7 14 22 29 37 44 52 59 67 74 82 89 97.  X is all ones and W[l, 0] = v[l] with
+    the other slots 0, so logit(l) = v[l]: a baseline -1 - l/1000 plus planted
+    values.  Expected answers are derived by hand from the bucket boundaries; a
+    partition with boundaries 7j, a ceil-based one, or one that loses the last
+    groups each drops a different planted label."""
+    n_groups, G, k, d, nb, K, Kp = 97, 4, 2, 8, 13, 5, 2
+    L = n_groups * G
+    idx = np.tile(np.array([0, 5], dtype=np.int32), (n_groups, 1))
+    v = -1.0 - np.arange(L) / 1000.0
+    planted = {85: 10.0, 87: 9.0,   # group 21, last group of bucket 2 = [14, 22)
+               88: 8.0,             # group 22, first group of bucket 3
+               386: 7.0,            # group 96, last group of the last bucket
+               0: 6.0,              # group 0
+               58: 5.0}             # group 14, first group of bucket 2: third best there, dropped
+    for l, val in planted.items():
+        v[l] = val
+    W = np.zeros((L, k), dtype=np.float64)
+    W[:, 0] = v
+    X = np.stack([np.ones(d), -np.ones(d)])
+    vals, ids = O.topk(X, W, idx, G, K, Kp, nb)
+    # row 0: bucket 2 keeps 10 and 9 (5 is its third), bucket 3 keeps 8, the last
+    # bucket 7, bucket 0 keeps 6
+    assert ids[0].tolist() == [85, 87, 88, 386, 0]
+    assert vals[0].tolist() == [10.0, 9.0, 8.0, 7.0, 6.0]
+    # row 1: logits -v, so larger labels rank first (the planted ones are now far
+    # below).  Each bucket passes its two largest labels: the last bucket
+    # (labels 356..387, 386 planted) passes 387 and 385, bucket 11 (labels
+    # 328..355) passes 355 and 354, bucket 10 (labels 296..327) passes 327.
+    assert ids[1].tolist() == [387, 385, 355, 354, 327]
+    np.testing.assert_allclose(vals[1], 1.0 + np.array([387, 385, 355, 354, 327]) / 1000.0, rtol=0, atol=1e-15)
