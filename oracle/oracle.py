@@ -179,6 +179,30 @@ def bce_loss(X, W, idx, G: int, row_ptr, ids, scale: float) -> float:
                                       _ptr(row_ptr), _ptr(ids), scale))
 
 
+# ------------------------------------------------------- optimizer update
+def sgd_update(W, M, dW64, lr: float, momentum: float):
+    """One step of SGD with heavy-ball momentum on the tail weights, in fp64:
+    M' = momentum * M + dW and W' = W - lr * M' (momentum = 0: M' = dW, W' =
+    W - lr * dW).  W and M are fp32, bf16 bits or fp64 (M may be None when
+    momentum is 0); returns (W', M') as float64.  This is the update the fused
+    step applies to each group's weights while its dW is still on chip; the
+    training loop it serves is the one of the HASTE summary page's experiments
+    (the page names no optimizer: plain SGD with momentum is this library's
+    choice)."""
+    W64 = to_f64(np.asarray(W))
+    M64 = np.zeros_like(W64) if M is None else to_f64(np.asarray(M))
+    M_new = momentum * M64 + dW64
+    return W64 - lr * M_new, M_new
+
+
+def bce_step_sgd(X, W, M, idx, G: int, row_ptr, ids, scale: float, lr: float, momentum: float):
+    """Fused tail step with the update: (loss, dX, W', M') in fp64; dX uses the
+    weights before the update."""
+    loss, _, dW, dX = bce_step(X, W, idx, G, row_ptr, ids, scale)
+    W_new, M_new = sgd_update(W, M, dW, lr, momentum)
+    return loss, dX, W_new, M_new
+
+
 # ------------------------------------------------ sampled single-output checks
 def logits_at(X, W, idx, G, bs, ls) -> np.ndarray:
     X, W, idx = _c(X), _c(W), _c(idx, np.int32)

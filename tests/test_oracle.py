@@ -311,6 +311,52 @@ def test_bce_loss_alone_matches_the_pinned_step_and_closed_forms():
     assert math.isclose(got, 0.5 * B * n_groups * G * math.log(2.0), rel_tol=1e-14)
 
 
+# ------------------------------------------------------- optimizer update
+def test_sgd_update_matches_torch_sgd_over_three_steps():
+    """The update equals torch.optim.SGD (momentum, no dampening, no Nesterov) on
+    the same gradients, step after step (the momentum buffer starts at zero)."""
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(3)
+    W = rng.normal(size=(12, 8))
+    grads = [rng.normal(size=(12, 8)) for _ in range(3)]
+    for lr, mu in ((0.1, 0.9), (0.5, 0.0), (0.03, 0.5)):
+        p = torch.nn.Parameter(torch.tensor(W, dtype=torch.float64))
+        opt = torch.optim.SGD([p], lr=lr, momentum=mu)
+        Wo, Mo = W.copy(), np.zeros_like(W)
+        for g in grads:
+            p.grad = torch.tensor(g, dtype=torch.float64)
+            opt.step()
+            Wo, Mo = O.sgd_update(Wo, Mo if mu else None, g, lr, mu)
+        np.testing.assert_allclose(Wo, p.detach().numpy(), rtol=1e-13, atol=1e-15)
+
+
+def test_sgd_update_special_cases():
+    rng = np.random.default_rng(4)
+    W, M, g = rng.normal(size=(5, 4)), rng.normal(size=(5, 4)), rng.normal(size=(5, 4))
+    W1, M1 = O.sgd_update(W, M, g, 0.0, 0.7)           # lr = 0: weights unchanged
+    assert np.array_equal(W1, W) and np.allclose(M1, 0.7 * M + g, rtol=0, atol=1e-15)
+    W2, M2 = O.sgd_update(W, None, g, 0.25, 0.0)       # no momentum: W - lr g
+    assert np.array_equal(M2, g) and np.allclose(W2, W - 0.25 * g, rtol=0, atol=1e-15)
+    Wb = I.make_normal((5, 4), 1.0, 4, 2, "bf16")       # bf16 bits widen exactly
+    W3, _ = O.sgd_update(Wb, None, np.zeros((5, 4)), 3.0, 0.0)
+    assert np.array_equal(W3, O.to_f64(Wb))
+
+
+def test_fused_step_with_update_is_step_then_update():
+    """dX uses the weights before the update; W' follows from the step's dW."""
+    B, d, n_groups, G, k = 6, 40, 7, 4, 8
+    idx = I.make_idx(n_groups, k, d, 8)
+    X = I.make_normal((B, d), 1.0, 8, 1, "f32")
+    W = I.make_normal((n_groups * G, k), 0.5, 8, 2, "f32")
+    M = I.make_normal((n_groups * G, k), 0.1, 8, 4, "f32")
+    rp, ids = I.make_zipf_positives(B, n_groups * G, 3, 1.0, 8)
+    loss, dX, W1, M1 = O.bce_step_sgd(X, W, M, idx, G, rp, ids, 1.0 / B, 0.2, 0.9)
+    r_loss, _, dW, r_dX = O.bce_step(X, W, idx, G, rp, ids, 1.0 / B)
+    assert loss == r_loss and np.array_equal(dX, r_dX)
+    np.testing.assert_allclose(M1, 0.9 * M.astype(np.float64) + dW, rtol=1e-14, atol=1e-15)
+    np.testing.assert_allclose(W1, W.astype(np.float64) - 0.2 * M1, rtol=1e-14, atol=1e-15)
+
+
 # ------------------------------------------------------------------- head
 def test_head_is_the_dense_special_case_of_the_sparse_layer():
     """A dense head over H labels is one group of G = H labels with k = d."""
