@@ -8,13 +8,17 @@ the C ABI of libhaste.so.  The fan-in plan is built once (it belongs to the
 sparsity pattern, not to the batch) and stays outside the timed region.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--config 670k] [--impl reference]
+                  [--more 8.6m,3m,sweep16,sweep32,sweep64]
 
-Default workload: the 670K-label tail (B=256, d=768, L=670,208 in groups of
+Headline workload: the 670K-label tail (B=256, d=768, L=670,208 in groups of
 G=32, k=128, bf16, 4,096 head labels, 5 Zipf(1.0) positives per sample).  Other
 workloads: 8.6m, 3m, sweep16/32/64 (forward + dW + dX with a given gradient),
-tiny.  Multi-GPU (torchrun) runs one independent replica of the layer per rank
-on its own batch (weak scaling, no collective on the data path); the timing is
-the max over ranks.  Prints one JSON line on rank 0.
+tiny.  A single-GPU run also measures the workloads listed by --more (default:
+the 8.6M and 3M steps and the three group sizes of the sweep) and reports them
+under "configs" in the same line.  Multi-GPU (torchrun) runs one independent
+replica of the layer per rank on its own batch (weak scaling, no collective on
+the data path); the timing is the max over ranks.  Prints one JSON line on
+rank 0.
 """
 from __future__ import annotations
 
@@ -109,7 +113,16 @@ def traffic_of(config, kernel):
         return None, "no capture of this kernel"
     if source_digest(kernel) != got[1]:
         return None, "kernel source changed since the capture"
-    return got[0], f"ncu capture, profiles/{KERNELS[kernel][1]}_{config}.md"
+    return got[0], f"ncu capture of {KERNELS[kernel][1]} at {config}"
+
+
+# A kernel timed inside a region shorter than this runs at the burst MMA rate;
+# longer regions settle at the sustained (power-capped) rate.
+SUSTAINED_AFTER_S = 2.0
+
+
+def use_sustained(region_ms):
+    return region_ms / 1e3 >= SUSTAINED_AFTER_S
 
 
 def roofline_of(flops, nbytes, ms, peaks, sustained=True):
@@ -316,7 +329,7 @@ def infer_topk(run, steps, warmup, peaks, K=5, kp=4):
     n_l, t_ms = prof.get("topk_score", (1, ms))
     flops = 2.0 * wl.B * wl.L * wl.k
     nbytes = wl.L * wl.k * 2 + 4 * wl.n_groups * wl.k + wl.B * wl.d * 2
-    rf = roofline_of(flops, nbytes, t_ms / max(n_l, 1), peaks)
+    rf = roofline_of(flops, nbytes, t_ms / max(n_l, 1), peaks, use_sustained(ms))
     rf["kernel"] = "topk_score"
     rf["traffic"], rf["traffic_src"] = traffic_of(wl.name, "topk_score")
     return {"metric": f"top-{K} tail scoring samples/s", "value": round(wl.B * steps / (ms / 1e3), 1),
@@ -383,6 +396,126 @@ def config_of(wl, l2_note):
     return c
 
 
+def l2_note(wl, dtype):
+    wb = wl.L * wl.k * (2 if dtype == "bf16" else 4) / 1e6
+    return (f"inputs larger than L2: W {wb:.0f} MB read and dW written every step (L2 126 MB)")
+
+
+def est_ms(run):
+    """One untimed step, timed roughly on the device: sizes the timed region."""
+    import torch
+    run.step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    run.step()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1)
+
+
+def sgd_variant(run, steps, warmup, peaks, lr=1e-3, momentum=0.9):
+    """The fused tail step with the SGD-with-momentum update in the step kernel
+    (haste_bce_step_sgd), alternating two weight buffers, device-timed.  W' and
+    the momentum replace the dW write: the step's compulsory bytes become W read,
+    W' written, momentum read and written."""
+    import torch
+    H, wl = run.H, run.wl
+    bufs = [run.W.clone(), torch.empty_like(run.W)]
+    M = torch.zeros_like(run.W)
+    state = {"i": 0}
+
+    def fn():
+        i = state["i"]
+        H.haste_bce_step_sgd(run.plan, run.X, bufs[i % 2], run.tp, run.ti, run.scale, run.loss[:1], lr, momentum,
+                             M, bufs[(i + 1) % 2], run.dX, run.ws)
+        state["i"] = i + 1
+
+    H.haste_profile_start()
+    ms = timed(fn, steps, warmup, False)
+    prof = H.haste_profile_stop()
+    if H.haste_device_status() != H.HASTE_OK:
+        raise SystemExit("device error word set during the fused-update timing")
+    tail_ms = sum(t for k, (n, t) in prof.items() if k.startswith("tail") or k in ("xt", "dx_reduce")) / steps
+    n_l, t_step = prof.get("tail_step", (1, 0.0))
+    e = 2
+    w = wl.L * wl.k * e
+    nbytes = 4 * w + 4 * wl.n_groups * wl.k + wl.B * wl.d * e      # W, W', momentum in and out, idx, X
+    rf = roofline_of(4.0 * wl.B * wl.L * wl.k, nbytes, t_step / max(n_l, 1), peaks, use_sustained(ms))
+    rf["kernel"] = "tail_step"
+    del bufs, M
+    return {"call": "haste_bce_step_sgd", "lr": lr, "momentum": momentum, "steps": steps,
+            "tail_ms_per_step": round(tail_ms, 4), "samples_per_s": round(wl.B / (tail_ms / 1e3), 1),
+            "step_kernel_ms": round(t_step / max(n_l, 1), 4), "roofline": rf}
+
+
+def replan_timing(run, frac=0.01, reps=5):
+    """Device re-plan after rewiring a fraction of the groups (haste_plan_update):
+    the changed rows are copied to the device and the inverse map is rebuilt
+    there.  The new rows are other groups' rows (valid sets), so the timing sees
+    a real rebuild.  Device-timed with CUDA events around the call, H2D included."""
+    import numpy as np
+    import torch
+    wl, plan = run.wl, run.plan
+    rng = np.random.default_rng(1)
+    n = max(1, int(frac * wl.n_groups))
+    groups = np.sort(rng.choice(wl.n_groups, n, replace=False)).astype(np.int32)
+    rows = run.inp.idx[rng.permutation(groups)]
+    times = []
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record()
+        plan.update(groups, rows)
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+        plan.update(groups, run.inp.idx[groups])          # back to the original sets
+        torch.cuda.synchronize()
+    return {"call": "haste_plan_update", "groups_changed": n, "ms": round(statistics.median(times), 4),
+            "full_plan_build_s": round(run.plan_s, 3)}
+
+
+def measure(run, steps, warmup, dist, peaks):
+    """Device-timed steps of one workload with the per-kernel profile, the
+    dominant kernel's roofline, the whole tail's roofline and the clocks seen."""
+    import torch
+    H, wl = run.H, run.wl
+    uuid = "GPU-" + str(torch.cuda.get_device_properties(torch.cuda.current_device()).uuid)
+    clk = Clocks(uuid)
+    time.sleep(0.2)
+    for _ in range(warmup):
+        run.step()
+    torch.cuda.synchronize()
+    H.haste_profile_start()
+    clk.mark()
+    ms = timed(run.step, steps, 0, dist)
+    clk.mark()
+    prof = H.haste_profile_stop()
+    clocks = clk.stop()
+    if H.haste_device_status() != H.HASTE_OK:
+        raise SystemExit("device error word set during the timed region")
+    sustained = use_sustained(ms)
+    work = algorithmic(wl)
+    dom = max((k for k in prof if k in work), key=lambda k: prof[k][1])
+    n_l, tot_ms = prof[dom]
+    rf = roofline_of(work[dom][0], work[dom][1], tot_ms / n_l, peaks, sustained)
+    rf["kernel"] = dom
+    rf["ms_per_launch"] = round(tot_ms / n_l, 4)
+    rf["peak_src"] = (f"{peaks['src']} ({('sustained' if sustained else 'burst') if rf['bound'] == 'tensor' else 'copy'}"
+                      f"; timed region {ms / 1e3:.2f} s)")
+    rf["traffic"], rf["traffic_src"] = traffic_of(wl.name, dom)
+    tail_ms = sum(prof[k][1] for k in prof if k.startswith("tail") or k in ("xt", "dx_reduce")) / steps
+    tail_rf = roofline_of(work["tail"][0], work["tail"][1], tail_ms, peaks, sustained)
+    total = sum(x[1] for x in prof.values())
+    return {"ms": ms, "prof": prof, "clocks": clocks, "roofline": rf,
+            "tail": {"ms_per_step": round(tail_ms, 4), "samples_per_s": round(wl.B / (tail_ms / 1e3), 1),
+                     "roofline": tail_rf},
+            "kernels": {k: {"launches": n, "ms_per_launch": round(t / n, 4), "share": round(t / total, 4)}
+                        for k, (n, t) in prof.items()},
+            "launches": sum(n for n, _ in prof.values())}
+
+
 # -------------------------------------------------------------------- main
 def main():
     ap = argparse.ArgumentParser()
@@ -393,6 +526,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget-s", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--more", default="8.6m,3m,sweep16,sweep32,sweep64",
+                    help="further workloads measured after the headline one (single GPU only; '' for none)")
+    ap.add_argument("--more-budget-ms", type=float, default=400.0, help="timed device time per further workload")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -444,21 +580,8 @@ def main():
     peaks = _peaks()
     run = Runner(wl, seed=rank)       # each rank: its own batch, its own replica
 
-    # device-resident timing
-    uuid = "GPU-" + str(torch.cuda.get_device_properties(torch.cuda.current_device()).uuid)
-    clk = Clocks(uuid)
-    time.sleep(0.2)
-    for _ in range(args.warmup):
-        run.step()
-    torch.cuda.synchronize()
-    H.haste_profile_start()
-    clk.mark()
-    ms = timed(run.step, args.steps, 0, dist)
-    clk.mark()
-    prof = H.haste_profile_stop()
-    clocks = clk.stop()
-    if H.haste_device_status() != H.HASTE_OK:
-        raise SystemExit("device error word set during the timed region")
+    res = measure(run, args.steps, args.warmup, dist, peaks)
+    ms, prof, clocks = res["ms"], res["prof"], res["clocks"]
 
     # end to end through the public API with host buffers
     run.e2e_setup()
@@ -466,40 +589,51 @@ def main():
 
     inference = infer_topk(run, args.steps, args.warmup, peaks) if wl.dtype == "bf16" and wl.B <= 256 else None
 
-    launches = sum(n for n, _ in prof.values())
-    work = algorithmic(wl)
-    dom = max((k for k in prof if k in work), key=lambda k: prof[k][1])
-    n_l, tot_ms = prof[dom]
-    rf = roofline_of(work[dom][0], work[dom][1], tot_ms / n_l, peaks)
-    rf["kernel"] = dom
-    rf["ms_per_launch"] = round(tot_ms / n_l, 4)
-    rf["peak_src"] = f"{peaks['src']} ({'sustained' if rf['bound'] == 'tensor' else 'copy'})"
-    rf["traffic"], rf["traffic_src"] = traffic_of(args.config, dom)
-    tail_ms = sum(prof[k][1] for k in prof if k.startswith("tail") or k in ("xt", "dx_reduce")) / args.steps
-    tail_rf = roofline_of(work["tail"][0], work["tail"][1], tail_ms, peaks)
-
     value = job_value(world, wl.B, args.steps, ms)
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": dtype, "data": "synthetic",
-        "config": config_of(wl, f"inputs larger than L2: W {wl.L * wl.k * (2 if dtype == 'bf16' else 4) / 1e6:.0f} MB "
-                                f"read and dW written every step (L2 126 MB)"),
-        "roofline": rf,
-        "tail": {"ms_per_step": round(tail_ms, 4), "samples_per_s": round(wl.B / (tail_ms / 1e3), 1),
-                 "roofline": tail_rf},
-        "kernels": {k: {"launches": n, "ms_per_launch": round(t / n, 4), "share": round(t / sum(
-            x[1] for x in prof.values()), 4)} for k, (n, t) in prof.items()},
+        "config": config_of(wl, l2_note(wl, dtype)),
+        "roofline": res["roofline"],
+        "tail": res["tail"],
+        "kernels": res["kernels"],
         "e2e": {"value": round(job_value(world, wl.B, args.steps, ms_e2e), 1), "unit": UNIT,
                 "h2d_bytes_per_step": run.h2d, "d2h_bytes_per_step": run.d2h},
-        "gpu_launches": launches,
+        "gpu_launches": res["launches"],
         "clocks": clocks,
         "plan_build_s": round(run.plan_s, 3),
         "inference": inference,
         "index_bytes": run.plan.info()[0],
     }
+    if wl.fused and wl.dtype == "bf16" and wl.B <= 256:
+        line["fused_update"] = sgd_variant(run, args.steps, args.warmup, peaks)
+        line["replan"] = replan_timing(run)
+    inp = run.inp
+    if world == 1 and args.more:
+        line["configs"] = {}
+        del run
+        torch.cuda.empty_cache()
+        for name in [c for c in args.more.split(",") if c and c != args.config]:
+            wlx = I.WORKLOADS[name]
+            rx = Runner(wlx, seed=rank)
+            steps = max(5, min(args.steps, int(round(args.more_budget_ms / max(est_ms(rx), 1e-3)))))
+            rr = measure(rx, steps, args.warmup, False, peaks)
+            line["configs"][name] = {
+                "config": config_of(wlx, l2_note(wlx, dtype)), "steps": steps,
+                "ms_per_step": round(rr["ms"] / steps, 4),
+                "samples_per_s": round(wlx.B * steps / (rr["ms"] / 1e3), 1),
+                "roofline": rr["roofline"], "tail": rr["tail"], "kernels": rr["kernels"],
+                "gpu_launches": rr["launches"], "clocks": rr["clocks"], "plan_build_s": round(rx.plan_s, 3),
+                "index_bytes": rx.plan.info()[0]}
+            if wlx.fused and wlx.dtype == "bf16" and wlx.B <= 256:
+                line["configs"][name]["fused_update"] = sgd_variant(rx, steps, args.warmup, peaks)
+                line["configs"][name]["replan"] = replan_timing(rx)
+            rx.plan.close()
+            del rx
+            torch.cuda.empty_cache()
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(run.inp, args.cpu_budget_s)
+        line["cpu_baseline"] = cpu_baseline(inp, args.cpu_budget_s)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist:

@@ -74,19 +74,17 @@ def make_idx(n_groups: int, k: int, d: int, seed: int = 0, *, stream: int = _T_I
 
 def make_normal(shape, std: float, seed: int, tensor_id: int, dtype: str) -> np.ndarray:
     """N(0, std^2) in fp32, returned as fp32 or as bf16 bits (uint16)."""
+    if dtype not in ("bf16", "f32"):
+        raise ValueError(dtype)
     rng = _rng(seed, tensor_id)
     n = int(np.prod(shape))
-    out32 = np.empty(n, dtype=np.float32)
+    out = np.empty(n, dtype=np.uint16 if dtype == "bf16" else np.float32)
     step = 1 << 24
-    for i in range(0, n, step):
+    for i in range(0, n, step):   # one chunk at a time: no full-size fp32 temporaries
         j = min(n, i + step)
-        out32[i:j] = rng.standard_normal(j - i, dtype=np.float32) * np.float32(std)
-    out32 = out32.reshape(shape)
-    if dtype == "bf16":
-        return f32_to_bf16_bits(out32)
-    if dtype == "f32":
-        return out32
-    raise ValueError(dtype)
+        v = rng.standard_normal(j - i, dtype=np.float32) * np.float32(std)
+        out[i:j] = f32_to_bf16_bits(v) if dtype == "bf16" else v
+    return out.reshape(shape)
 
 
 def make_zipf_positives(B: int, n_ids: int, p: int, alpha: float, seed: int,

@@ -59,7 +59,7 @@ def test_traffic_is_reported_only_for_the_captured_source(monkeypatch):
     assert digest is not None and len(digest) == 16
     monkeypatch.setattr(bench, "TRAFFIC", {("670k", "tail_step"): (123e6, digest)})
     got, src = bench.traffic_of("670k", "tail_step")
-    assert got == 123e6 and "profiles/k_step2_670k.md" in src
+    assert got == 123e6 and src == "ncu capture of k_step2 at 670k"
     # a capture taken on another version of the kernel's source is not reported
     monkeypatch.setattr(bench, "TRAFFIC", {("670k", "tail_step"): (123e6, "0" * 16)})
     got, src = bench.traffic_of("670k", "tail_step")
@@ -74,6 +74,13 @@ def test_every_timed_kernel_has_a_source_file():
         assert os.path.exists(os.path.join(bench.CSRC, src)), kernel
         with open(os.path.join(bench.CSRC, src)) as fh:
             assert name in fh.read(), (kernel, name)
+
+
+def test_peak_choice_follows_the_timed_region():
+    # kernels timed inside a short region run at the burst rate, long ones at the
+    # sustained (power-capped) rate
+    assert not bench.use_sustained(140.0)
+    assert bench.use_sustained(bench.SUSTAINED_AFTER_S * 1e3)
 
 
 def test_job_value_counts_every_rank():
