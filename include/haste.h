@@ -36,8 +36,8 @@
  *     hanging; haste_device_status() synchronises and reports it.
  *   - Supported by the GPU path: k*elem % 128 == 0 (k % 64 for bf16, k % 32 for
  *     fp32), k <= 256, G % 16 == 0, 16 <= G <= 128, L*elem % 16 == 0, B <= 512;
- *     head: H*elem and d*elem multiples of 16 bytes.
- *     B <= 512.  Other shapes return HASTE_ERR_UNSUPPORTED_SHAPE.
+ *     head: H*elem and d*elem multiples of 16 bytes.  Other shapes return
+ *     HASTE_ERR_UNSUPPORTED_SHAPE.
  *   - Results are deterministic: repeated calls give identical bits (fixed-order
  *     reductions, no floating-point atomics).
  */
@@ -92,6 +92,18 @@ haste_status_t haste_device_status(haste_stream_t stream);
  * usable.  No GPU fault is involved. */
 haste_status_t haste_selftest_wait_timeout(haste_stream_t stream);
 
+/* Limit, in ns, of the waits between the warps of the pipelined kernels (a
+ * producer waiting for a free ring stage, a consumer for a full one) on the
+ * current device, for kernels launched after the call; 0 restores the default of
+ * 2 s, larger values are refused (HASTE_ERR_INVALID_ARG).  A wait that runs out
+ * sets the device error word and the kernel unwinds: its results are then
+ * undefined and haste_device_status() returns HASTE_ERR_TIMEOUT.  Waits for a
+ * kernel's own copies or MMAs in flight keep the 2 s limit, so that no kernel
+ * exits while they can still write its memory.  Meant for failure-detection
+ * tests (a very short limit forces the abort paths); not thread-safe against
+ * concurrent launches. */
+haste_status_t haste_set_wait_limit_ns(uint64_t ns);
+
 /* Per-kernel timing without a profiler.  Between haste_profile_start() and
  * haste_profile_stop(), every kernel the library launches is bracketed by CUDA
  * events recorded on its launch stream.  haste_profile_stop() waits for those
@@ -119,24 +131,54 @@ int32_t haste_profile_stop(haste_kernel_time_t* out, int32_t max_entries);
 haste_status_t haste_plan_inverse_host(const int32_t* idx, int64_t n_groups, int32_t k, int32_t d,
                                        int32_t* inv_off, int32_t* inv_ent);
 
-/* Build a plan: validate idx (host [n_groups*k]), build the inverse map, copy
- * idx, inv_off and inv_ent to the current device (stream-ordered copies; the
- * call returns after they complete).  *out receives the new plan. */
+/* Build a plan: validate idx (host [n_groups*k]), copy it to the current device
+ * and build the inverse map there (the stable counting sort described at
+ * haste_plan_inverse_host, on the device; for d above about 57,000 features it
+ * is built on the host and copied).  The call returns after the work completes.
+ * *out receives the new plan, which belongs
+ * to that device: calls made while another device is current are refused with
+ * HASTE_ERR_INVALID_ARG.  Source: Methodology 1, structure (one index set I_g
+ * shared by the G labels of a group) and memory efficiency (indices stored once
+ * per group, not once per label). */
 haste_status_t haste_plan(haste_plan_t* out, const int32_t* idx, int64_t n_groups, int32_t G, int32_t k,
                           int32_t d, haste_stream_t stream);
+
+/* Rewire the fan-in sets of some groups, for dynamic sparse training (the
+ * HASTE page's title: the index sets change during training; how they change is
+ * the caller's rule): the index rows of the n_changed groups listed in groups
+ * (host, ascending, distinct, in [0, n_groups)) become rows (host
+ * [n_changed * k], each row strictly increasing in [0, d)), and the inverse map
+ * is rebuilt on the device.  Only the changed rows cross PCIe.  Validation as
+ * haste_plan (HASTE_ERR_INDEX_* for a bad row, HASTE_ERR_INVALID_ARG for bad
+ * group ids) happens before anything changes.  The update is ordered on
+ * `stream`: later calls on that stream see the new sets; work on other streams
+ * that uses the plan must be ordered by the caller.  The host arrays may be
+ * reused when the call returns.  A plan whose inverse map was built on the host
+ * (very large d) returns HASTE_ERR_UNSUPPORTED_SHAPE.  n_changed = 0 is a no-op.
+ * The weights of a rewired group keep their slots: the caller resets or carries
+ * over W and dW rows of the changed groups as its rule says. */
+haste_status_t haste_plan_update(haste_plan_t plan, const int32_t* groups, int64_t n_changed, const int32_t* rows,
+                                 haste_stream_t stream);
 
 /* Free a plan's device and host memory (synchronous).  NULL is accepted. */
 haste_status_t haste_plan_destroy(haste_plan_t plan);
 
 /* Index store of the plan: index_bytes = 4*n_groups*k (one int32 per group and
- * slot, against 4*L*k for per-label fan-in); inverse_bytes = 4*(d+1+n_groups*k). */
+ * slot, against 4*L*k for per-label fan-in); inverse_bytes = 4*(d+1+n_groups*k).
+ * Source: Methodology 1, memory efficiency (the saving of storing the fan-in
+ * indices per group). */
 haste_status_t haste_plan_info(haste_plan_t plan, int64_t* index_bytes, int64_t* inverse_bytes);
 
 /* Copy the plan's DEVICE arrays back to host buffers (synchronous): idx
- * [n_groups*k], inv_off [d+1], inv_ent [n_groups*k].  Any pointer may be NULL. */
+ * [n_groups*k], inv_off [d+1], inv_ent [n_groups*k].  Any pointer may be NULL.
+ * For bit-exact checks of the plan (Methodology 1, structure and memory
+ * efficiency). */
 haste_status_t haste_plan_export(haste_plan_t plan, int32_t* idx, int32_t* inv_off, int32_t* inv_ent);
 
-/* Workspace bytes that every sparse-tail call below needs at batch B. */
+/* Workspace bytes that every sparse-tail call below needs at batch B (0 for a
+ * NULL plan, B <= 0 or a plan of another device).  The workspace holds X^T, the
+ * dX pass's partial sums and the fused step's gradient buffer: the staging that
+ * Methodology 1's gather-once, dense-product scheme needs on this GPU. */
 size_t haste_workspace_size(haste_plan_t plan, int32_t B, haste_dtype_t dtype);
 
 /* ------------------------------------------------------------- sparse tail --- */
@@ -147,13 +189,18 @@ size_t haste_workspace_size(haste_plan_t plan, int32_t B, haste_dtype_t dtype);
 haste_status_t haste_forward(haste_plan_t plan, int32_t B, haste_dtype_t dtype, const void* X, const void* W,
                              void* logits, void* ws, size_t ws_bytes, haste_stream_t stream);
 
-/* dW[g*G+j, s] = sum_b dY[b, g*G+j] * X[b, idx[g,s]], dW in the input dtype. */
+/* dW[g*G+j, s] = sum_b dY[b, g*G+j] * X[b, idx[g,s]], dW in the input dtype.
+ * Source: Methodology 1 (the gathered inputs X[:, I_g] are shared by the G labels
+ * of a group, so dW_g = dY_g^T . X[:, I_g] is one dense product per group) and
+ * Experimental results (the backward pass's speed-up over per-label fan-in). */
 haste_status_t haste_backward_dw(haste_plan_t plan, int32_t B, haste_dtype_t dtype, const void* X,
                                  const void* dY, void* dW, void* ws, size_t ws_bytes, haste_stream_t stream);
 
 /* dX[b, f] (+)= sum over the (g, s) with idx[g,s] == f, in ascending g, of
  * sum_j dY[b, g*G+j] * W[g*G+j, s]; fp32 output.  accumulate = 0 overwrites dX,
- * 1 adds into it.  Features in no group receive exactly 0. */
+ * 1 adds into it.  Features in no group receive exactly 0.  Source: Methodology 1
+ * (a group's G labels scatter into the same k features I_g, so its contribution
+ * dY_g . W_g lands in dX[:, I_g]) and Experimental results (backward speed-up). */
 haste_status_t haste_backward_dx(haste_plan_t plan, int32_t B, haste_dtype_t dtype, const void* W,
                                  const void* dY, float* dX, int accumulate, void* ws, size_t ws_bytes,
                                  haste_stream_t stream);
@@ -181,7 +228,9 @@ haste_status_t haste_backward_dx(haste_plan_t plan, int32_t B, haste_dtype_t dty
 haste_status_t haste_backward_dx_noalloc(haste_plan_t plan, int32_t B, haste_dtype_t dtype, const void* W,
                                          const void* dY, float* dX, int accumulate, haste_stream_t stream);
 
-/* Fused tail training step (logits never reach global memory):
+/* Fused tail training step (logits never reach global memory), the forward and
+ * backward of Methodology 1 with the loss in between (Experimental results: the
+ * forward and backward speed-ups, and the training-memory saving):
  *   z = forward(X, W);  y[b,l] = 1 iff l is in tail_pos row b;
  *   dY = grad_scale * (sigmoid(z) - y)   (rounded to the input dtype);
  *   *loss = grad_scale * sum_{b,l} (softplus(z) - z*y)   (if loss != NULL, device fp32);
@@ -192,6 +241,27 @@ haste_status_t haste_backward_dx_noalloc(haste_plan_t plan, int32_t B, haste_dty
 haste_status_t haste_bce_step(haste_plan_t plan, int32_t B, haste_dtype_t dtype, const void* X, const void* W,
                               haste_targets_t tail_pos, float grad_scale, float* loss, void* dW, float* dX,
                               int accumulate, void* ws, size_t ws_bytes, haste_stream_t stream);
+
+/* Fused tail training step with the optimizer update fused into it: as
+ * haste_bce_step, but instead of writing dW the step kernel updates each group's
+ * weights while its dW is still on chip (SGD with heavy-ball momentum):
+ *   M' = momentum * M + dW   (M' = dW when momentum == 0),
+ *   W_out = W - lr * M'.
+ * W is read, not written: the dX pass of the same call still needs it, so W_out
+ * must be a different buffer (callers alternate two weight buffers).  M [L, k]
+ * holds the momentum in W's dtype and is updated in place; it may be NULL when
+ * momentum == 0; start it at zero.  dX and the loss are those of haste_bce_step
+ * (computed with W).  Compared with haste_bce_step followed by a separate
+ * update, the dW write and the update pass's reads of W and dW never happen.
+ * Supported: bf16, G in {16, 32, 64}, k in {64, 128}, B <= 256; other shapes
+ * return HASTE_ERR_UNSUPPORTED_SHAPE.  Source: Methodology 1 (the per-group dW
+ * product) and the training loop of Experimental results (training memory);
+ * the page names no optimizer, plain SGD with momentum is this library's
+ * choice. */
+haste_status_t haste_bce_step_sgd(haste_plan_t plan, int32_t B, haste_dtype_t dtype, const void* X, const void* W,
+                                  haste_targets_t tail_pos, float grad_scale, float* loss, float lr, float momentum,
+                                  void* M, void* W_out, float* dX, int accumulate, void* ws, size_t ws_bytes,
+                                  haste_stream_t stream);
 
 /* ----------------------------------------------------- top-k scoring --- */
 

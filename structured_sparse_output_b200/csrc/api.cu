@@ -20,7 +20,10 @@
 #include "tail.cu"
 #include "tail_v2.cu"
 #include "dx_band.cu"
+#include "dx_z.cu"
+#include "tail_given.cu"
 #include "topk.cu"
+#include "plan.cu"
 
 using namespace haste;
 
@@ -31,6 +34,9 @@ struct haste_plan_s {
   int32_t* idx_d;
   int32_t* inv_off_d;
   int32_t* inv_ent_d;
+  int32_t* scratch_d;  // counting-sort scratch of the device build (NULL: built on the host)
+  int32_t* upd_d;      // staging of haste_plan_update: changed group ids and rows
+  size_t upd_cap;      // ints of upd_d
 };
 
 namespace {
@@ -123,26 +129,28 @@ class ProfScope {
   cudaEvent_t a_ = nullptr;
 };
 
-// Tiling of the dX pass: feature bands (at most 256 features, the MMA N, in the
-// pipelined kernel; sized so the fp32 band accumulator fits in shared memory in
-// the staged one); group chunks so that all CTAs are resident.  ns > 0: the
-// pipelined kernel with an ns-stage ring; ns = 0: the staged kernel.
+// Tiling of the dX pass.  ns > 0: the pipelined scatter kernel (k_dx_z) with an
+// ns-stage ring, one CTA per (group chunk, 128-row batch tile, feature part of
+// part_w features); ns = 0: the staged kernel, feature bands sized so the fp32
+// band accumulator fits in shared memory.  Group chunks: as many as keep every
+// CTA resident.
 struct DxTiling {
-  int band, n_bands, n_chunks, ns;
+  int band, n_bands, n_chunks, ns, n_parts, part_w;
 };
 
-// The warp-specialised TMA kernels cover bf16 with G in {16, 32, 64}, k in
-// {64, 128} and at most two 128-row batch tiles; other shapes run the staged
-// kernels of tail.cu.
+// The warp-specialised TMA kernels cover bf16 with G in {16, 32, 64} and k in
+// {64, 128}: the fused step kernel up to two 128-row batch tiles, the dX pass up
+// to four; other shapes run the staged kernels of tail.cu.
 bool use_v2(const haste_plan_s& p, int Bp, int elem) { return elem == 2 && tail2::supported(p.G, p.k, Bp); }
+bool use_dxz(const haste_plan_s& p, int Bp, int elem) { return elem == 2 && tail2::dxz_supported(p.G, p.k, Bp); }
 
 DxTiling dx_tiling(const haste_plan_s& p, int Bp, int elem, int sms, int smem_optin) {
   DxTiling t{};
   const int kHeadroom = 4096;  // static shared memory and launch reserve
   int per_chunk;
-  if (use_v2(p, Bp, elem) &&
-      tail2::dx_config(p.G, p.k, p.d, Bp, (size_t)smem_optin, kHeadroom, &t.band, &t.n_bands, &t.ns)) {
-    per_chunk = t.n_bands;  // a CTA covers every batch row of its band
+  if (use_dxz(p, Bp, elem) &&
+      tail2::dxz_config(p.G, p.k, p.d, (size_t)smem_optin, kHeadroom, &t.n_parts, &t.part_w, &t.ns)) {
+    per_chunk = (Bp / 128) * t.n_parts;
   } else {
     const long avail = (long)smem_optin - (long)tail::smem_dx(elem, p.k, p.G, 0) - kHeadroom;
     int band = (int)std::min<long>(256, avail / 512);
@@ -183,8 +191,20 @@ TailWs tail_ws(const haste_plan_s& p, int B, int elem, const DxTiling& t) {
   return w;
 }
 
+// A plan's arrays live on the device that was current when it was built; a call
+// on another device would read them through peer access or fault.
+haste_status_t check_plan_device(const haste_plan_s* p) {
+  if (!p) return fail(HASTE_ERR_INVALID_ARG, "plan is NULL");
+  int dev = -1;
+  HASTE_CUDA(cudaGetDevice(&dev));
+  if (dev != p->device)
+    return fail(HASTE_ERR_INVALID_ARG, "the plan was built on device %d, but device %d is current", p->device, dev);
+  return HASTE_OK;
+}
+
 haste_status_t check_tail(const haste_plan_s* p, int B, haste_dtype_t dt, const DeviceInfo& di) {
   if (!p) return fail(HASTE_ERR_INVALID_ARG, "plan is NULL");
+  if (haste_status_t st = check_plan_device(p)) return st;
   if (dt != HASTE_F32 && dt != HASTE_BF16) return fail(HASTE_ERR_INVALID_ARG, "unknown dtype %d", (int)dt);
   if (B <= 0) return fail(HASTE_ERR_INVALID_ARG, "B must be positive (got %d)", B);
   const int E = elem_bytes(dt);
@@ -222,24 +242,22 @@ TailArgs make_args(const haste_plan_s& p, int B) {
   return a;
 }
 
-// dX pass through the pipelined bf16 kernel.  Element (b, g*G + j) of dY sits at
-// dY[g*gstride + b*rstride + j]: (G, L) for the caller's [B, L] gradient,
-// (Bp*G, G) for the fused step's group-major buffer.
-cudaError_t dx_v2(const haste_plan_s& p, int B, const void* W, const void* dY, int64_t gstride, int64_t rstride,
-                  float* part, const DxTiling& t, cudaStream_t s) {
-  v2::DxArgs a{};
+// dX pass through the pipelined bf16 kernel, from the caller's row-major [B, L]
+// gradient or from the fused step's group-major buffer [n_groups, Bp, G].
+cudaError_t dx_v2(const haste_plan_s& p, int B, const void* W, const void* dY, bool group_major, float* part,
+                  const DxTiling& t, cudaStream_t s) {
+  v2::DxzArgs a{};
   a.sh = make_args(p, B).sh;
   a.idx = p.idx_d;
   a.dY = static_cast<const __nv_bfloat16*>(dY);
   a.W = static_cast<const __nv_bfloat16*>(W);
   a.dX_part = part;
-  a.band = t.band;
-  a.n_bands = t.n_bands;
   a.n_chunks = t.n_chunks;
+  a.n_parts = t.n_parts;
+  a.part_w = t.part_w;
   a.ns = t.ns;
-  a.dy_gstride = gstride;
-  a.dy_rstride = rstride;
-  return tail2::launch_dx(p.G, p.k, a, dY, W, s);
+  a.dy_group_major = group_major ? 1 : 0;
+  return tail2::launch_dxz(p.G, p.k, a, dY, W, s);
 }
 
 template <typename T>
@@ -272,6 +290,44 @@ haste_status_t noalloc_scratch(void** out) {
   *out = g_noalloc_addr[dev];
   return HASTE_OK;
 }
+
+// Validation of index rows (host [n_rows, k]): the first offending element in
+// row-major order decides: out of [0, d) -> HASTE_ERR_INDEX_OUT_OF_RANGE, not
+// above its predecessor -> HASTE_ERR_INDEX_UNSORTED_OR_DUP.  `what` names the
+// rows in the message.  Split over threads by contiguous row ranges.
+haste_status_t validate_rows(const int32_t* idx, int64_t n_rows, int32_t k, int32_t d, const char* what) {
+  const unsigned hw = std::thread::hardware_concurrency();
+  const int nt = (int)std::min<int64_t>(std::max(1u, std::min(hw, 32u)), std::max<int64_t>(1, n_rows * k / (1 << 16)));
+  std::vector<int64_t> bad(nt, -1);
+  std::vector<int> code(nt, 0);
+  auto scan = [&](int t) {
+    for (int64_t r = n_rows * t / nt; r < n_rows * (t + 1) / nt; ++r) {
+      int32_t prev = -1;
+      for (int32_t s = 0; s < k; ++s) {
+        const int32_t f = idx[r * k + s];
+        if ((uint32_t)f >= (uint32_t)d || f <= prev) {
+          bad[t] = r * k + s;
+          code[t] = (uint32_t)f >= (uint32_t)d ? HASTE_ERR_INDEX_OUT_OF_RANGE : HASTE_ERR_INDEX_UNSORTED_OR_DUP;
+          return;
+        }
+        prev = f;
+      }
+    }
+  };
+  std::vector<std::thread> th;
+  for (int t = 1; t < nt; ++t) th.emplace_back(scan, t);
+  scan(0);
+  for (auto& x : th) x.join();
+  for (int t = 0; t < nt; ++t)
+    if (bad[t] >= 0)
+      return fail((haste_status_t)code[t], "%s element %lld (row %lld, slot %lld) is %s", what, (long long)bad[t],
+                  (long long)(bad[t] / k), (long long)(bad[t] % k),
+                  code[t] == HASTE_ERR_INDEX_OUT_OF_RANGE ? "out of [0, d)" : "not above its predecessor");
+  return HASTE_OK;
+}
+
+// The device build needs the d feature counters of a chunk in shared memory.
+bool device_build_fits(int d, int smem_optin) { return (size_t)d * 4 + 1024 <= (size_t)smem_optin; }
 
 }  // namespace
 
@@ -322,6 +378,14 @@ int32_t haste_profile_stop(haste_kernel_time_t* out, int32_t max_entries) {
   const int32_t n = (int32_t)agg.size();
   for (int32_t i = 0; out && i < n && i < max_entries; ++i) out[i] = agg[i];
   return n;
+}
+
+haste_status_t haste_set_wait_limit_ns(uint64_t ns) {
+  const uint64_t v = ns ? ns : kWaitLimitNs;
+  if (v > kWaitLimitNs) return fail(HASTE_ERR_INVALID_ARG, "wait limit %llu ns above the default %llu ns",
+                                    (unsigned long long)v, (unsigned long long)kWaitLimitNs);
+  HASTE_CUDA(cudaMemcpyToSymbol(g_wait_limit_ns, &v, sizeof v));
+  return HASTE_OK;
 }
 
 haste_status_t haste_selftest_wait_timeout(haste_stream_t stream) {
@@ -415,31 +479,91 @@ haste_status_t haste_plan(haste_plan_t* out, const int32_t* idx, int64_t n_group
   if (!out) return fail(HASTE_ERR_INVALID_ARG, "out is NULL");
   *out = nullptr;
   if (G <= 0) return fail(HASTE_ERR_INVALID_ARG, "G must be positive");
+  if (!idx) return fail(HASTE_ERR_INVALID_ARG, "NULL pointer");
+  if (n_groups <= 0 || k <= 0 || d <= 0) return fail(HASTE_ERR_INVALID_ARG, "n_groups, k and d must be positive");
   if (n_groups * (int64_t)G > 0x7fffffffffffLL) return fail(HASTE_ERR_INVALID_ARG, "L too large");
-  const int64_t n = n_groups * (int64_t)k;
-  std::vector<int32_t> off((size_t)std::max(d, 0) + 1), ent((size_t)std::max<int64_t>(n, 0));
-  haste_status_t st = haste_plan_inverse_host(idx, n_groups, k, d, off.data(), ent.data());
+  if (n_groups * (int64_t)k > 0x7fffffffLL) return fail(HASTE_ERR_UNSUPPORTED_SHAPE, "n_groups*k must fit in int32");
+  haste_status_t st = validate_rows(idx, n_groups, k, d, "idx");
   if (st != HASTE_OK) return st;
+  DeviceInfo di;
+  if ((st = device_info(di)) != HASTE_OK) return st;
+  const int64_t n = n_groups * (int64_t)k;
   haste_plan_s* p = new haste_plan_s{};
   p->n_groups = n_groups;
   p->G = G;
   p->k = k;
   p->d = d;
-  cudaGetDevice(&p->device);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e = cudaMalloc(&p->idx_d, n * 4);
+  const bool on_device = device_build_fits(d, di.smem_optin);
+  std::vector<int32_t> off, ent;
+  cudaError_t e = cudaGetDevice(&p->device);
+  if (e == cudaSuccess) e = cudaMalloc(&p->idx_d, n * 4);
   if (e == cudaSuccess) e = cudaMalloc(&p->inv_off_d, ((size_t)d + 1) * 4);
   if (e == cudaSuccess) e = cudaMalloc(&p->inv_ent_d, n * 4);
+  if (e == cudaSuccess && on_device) e = cudaMalloc(&p->scratch_d, plan::scratch_ints(n_groups, d) * 4);
   if (e == cudaSuccess) e = cudaMemcpyAsync(p->idx_d, idx, n * 4, cudaMemcpyHostToDevice, s);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(p->inv_off_d, off.data(), ((size_t)d + 1) * 4, cudaMemcpyHostToDevice, s);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(p->inv_ent_d, ent.data(), n * 4, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess && on_device) {
+    e = plan::build_inverse(p->idx_d, n_groups, k, d, p->scratch_d, p->inv_off_d, p->inv_ent_d, s);
+  } else if (e == cudaSuccess) {
+    // wide d: the inverse map is built on the host and uploaded
+    off.resize((size_t)d + 1);
+    ent.resize((size_t)n);
+    if ((st = haste_plan_inverse_host(idx, n_groups, k, d, off.data(), ent.data())) != HASTE_OK) {
+      cudaStreamSynchronize(s);
+      haste_plan_destroy(p);
+      return st;
+    }
+    e = cudaMemcpyAsync(p->inv_off_d, off.data(), ((size_t)d + 1) * 4, cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(p->inv_ent_d, ent.data(), n * 4, cudaMemcpyHostToDevice, s);
+  }
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) {
     haste_plan_destroy(p);
-    return cuda_fail(e, "plan upload");
+    return cuda_fail(e, "plan build");
   }
   *out = p;
   return HASTE_OK;
+}
+
+haste_status_t haste_plan_update(haste_plan_t p, const int32_t* groups, int64_t n_changed, const int32_t* rows,
+                                 haste_stream_t stream) {
+  haste_status_t st = check_plan_device(p);
+  if (st != HASTE_OK) return st;
+  if (n_changed < 0 || n_changed > p->n_groups) return fail(HASTE_ERR_INVALID_ARG, "n_changed out of [0, n_groups]");
+  if (n_changed == 0) return HASTE_OK;
+  if (!groups || !rows) return fail(HASTE_ERR_INVALID_ARG, "NULL pointer");
+  if (!p->scratch_d)
+    return fail(HASTE_ERR_UNSUPPORTED_SHAPE, "d=%d: the plan's inverse map is built on the host; rebuild the plan",
+                p->d);
+  for (int64_t i = 0; i < n_changed; ++i)
+    if (groups[i] < 0 || groups[i] >= p->n_groups || (i > 0 && groups[i] <= groups[i - 1]))
+      return fail(HASTE_ERR_INVALID_ARG, "groups[%lld] = %d: group ids must be ascending in [0, n_groups)",
+                  (long long)i, groups[i]);
+  if ((st = validate_rows(rows, n_changed, p->k, p->d, "rows")) != HASTE_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t need = (size_t)n_changed * (p->k + 1);
+  if (need > p->upd_cap) {
+    HASTE_CUDA(cudaStreamSynchronize(s));  // an earlier update may still read the old staging
+    cudaFree(p->upd_d);
+    p->upd_d = nullptr;
+    p->upd_cap = 0;
+    HASTE_CUDA(cudaMalloc(&p->upd_d, need * 4));
+    p->upd_cap = need;
+  }
+  int32_t* g_d = p->upd_d;
+  int32_t* r_d = p->upd_d + n_changed;
+  HASTE_CUDA(cudaMemcpyAsync(g_d, groups, (size_t)n_changed * 4, cudaMemcpyHostToDevice, s));
+  HASTE_CUDA(cudaMemcpyAsync(r_d, rows, (size_t)n_changed * p->k * 4, cudaMemcpyHostToDevice, s));
+  cudaError_t e;
+  {
+    ProfScope ps("plan_update", s);
+    const int64_t tot = n_changed * p->k;
+    plan::k_plan_set_rows<<<(unsigned)((tot + 255) / 256), 256, 0, s>>>(p->idx_d, p->k, g_d, r_d, n_changed);
+    e = cudaGetLastError();
+    if (e == cudaSuccess)
+      e = plan::build_inverse(p->idx_d, p->n_groups, p->k, p->d, p->scratch_d, p->inv_off_d, p->inv_ent_d, s);
+  }
+  return e == cudaSuccess ? HASTE_OK : cuda_fail(e, "haste_plan_update launch");
 }
 
 haste_status_t haste_plan_destroy(haste_plan_t p) {
@@ -447,6 +571,8 @@ haste_status_t haste_plan_destroy(haste_plan_t p) {
   cudaFree(p->idx_d);
   cudaFree(p->inv_off_d);
   cudaFree(p->inv_ent_d);
+  cudaFree(p->scratch_d);
+  cudaFree(p->upd_d);
   delete p;
   return HASTE_OK;
 }
@@ -459,7 +585,7 @@ haste_status_t haste_plan_info(haste_plan_t p, int64_t* index_bytes, int64_t* in
 }
 
 haste_status_t haste_plan_export(haste_plan_t p, int32_t* idx, int32_t* inv_off, int32_t* inv_ent) {
-  if (!p) return fail(HASTE_ERR_INVALID_ARG, "plan is NULL");
+  if (haste_status_t st = check_plan_device(p)) return st;
   const size_t n = (size_t)p->n_groups * p->k;
   if (idx) HASTE_CUDA(cudaMemcpy(idx, p->idx_d, n * 4, cudaMemcpyDeviceToHost));
   if (inv_off) HASTE_CUDA(cudaMemcpy(inv_off, p->inv_off_d, ((size_t)p->d + 1) * 4, cudaMemcpyDeviceToHost));
@@ -468,7 +594,7 @@ haste_status_t haste_plan_export(haste_plan_t p, int32_t* idx, int32_t* inv_off,
 }
 
 size_t haste_workspace_size(haste_plan_t p, int32_t B, haste_dtype_t dt) {
-  if (!p || B <= 0) return 0;
+  if (!p || B <= 0 || check_plan_device(p) != HASTE_OK) return 0;
   DeviceInfo di;
   if (device_info(di) != HASTE_OK) return 0;
   const int Bp = round_up(B, 128);
@@ -500,7 +626,21 @@ haste_status_t haste_forward(haste_plan_t p, int32_t B, haste_dtype_t dt, const 
   }
   if (e == cudaSuccess) {
     ProfScope ps("tail_forward", s);
-    e = dt == HASTE_BF16 ? tail::launch_forward<__nv_bfloat16>(a, di.sms, s) : tail::launch_forward<float>(a, di.sms, s);
+    const int Bp = a.sh.Bp, ns = tail3::stages(p->k, p->G, (size_t)di.smem_optin, 4096);
+    if (dt == HASTE_BF16 && tail3::supported(p->G, p->k, Bp) && ns > 0) {
+      v3::GivenArgs g{};
+      g.sh = a.sh;
+      g.idx = p->idx_d;
+      g.Xt = static_cast<const __nv_bfloat16*>(a.Xt);
+      g.W = static_cast<const __nv_bfloat16*>(W);
+      g.out = static_cast<__nv_bfloat16*>(logits);
+      g.n_chunks = (int)std::min<int64_t>(p->n_groups, std::max(1, di.sms / (Bp / 128)));
+      g.ns = ns;
+      e = tail3::launch_fwd(p->G, p->k, g, s);
+    } else {
+      e = dt == HASTE_BF16 ? tail::launch_forward<__nv_bfloat16>(a, di.sms, s)
+                           : tail::launch_forward<float>(a, di.sms, s);
+    }
   }
   return e == cudaSuccess ? HASTE_OK : cuda_fail(e, "haste_forward launch");
 }
@@ -529,8 +669,21 @@ haste_status_t haste_backward_dw(haste_plan_t p, int32_t B, haste_dtype_t dt, co
   }
   if (e == cudaSuccess) {
     ProfScope ps("tail_dw", s);
-    e = dt == HASTE_BF16 ? tail::launch_backward_dw<__nv_bfloat16>(a, di.sms, s)
-                         : tail::launch_backward_dw<float>(a, di.sms, s);
+    const int Bp = a.sh.Bp, ns = tail3::stages(p->k, p->G, (size_t)di.smem_optin, 4096);
+    if (dt == HASTE_BF16 && tail3::supported(p->G, p->k, Bp) && ns > 0) {
+      v3::GivenArgs g{};
+      g.sh = a.sh;
+      g.idx = p->idx_d;
+      g.Xt = static_cast<const __nv_bfloat16*>(a.Xt);
+      g.dY = static_cast<const __nv_bfloat16*>(dY);
+      g.out = static_cast<__nv_bfloat16*>(dW);
+      g.n_chunks = (int)std::min<int64_t>(p->n_groups, di.sms);
+      g.ns = ns;
+      e = tail3::launch_dw(p->G, p->k, g, s);
+    } else {
+      e = dt == HASTE_BF16 ? tail::launch_backward_dw<__nv_bfloat16>(a, di.sms, s)
+                           : tail::launch_backward_dw<float>(a, di.sms, s);
+    }
   }
   return e == cudaSuccess ? HASTE_OK : cuda_fail(e, "haste_backward_dw launch");
 }
@@ -558,7 +711,7 @@ haste_status_t haste_backward_dx(haste_plan_t p, int32_t B, haste_dtype_t dt, co
   {
     ProfScope ps("tail_dx", s);
     if (t.ns > 0)
-      e = dx_v2(*p, B, W, dY, p->G, a.sh.L, a.dX_part, t, s);
+      e = dx_v2(*p, B, W, dY, false, a.dX_part, t, s);
     else
       e = dt == HASTE_BF16 ? tail::launch_backward_dx<__nv_bfloat16>(a, false, s)
                            : tail::launch_backward_dx<float>(a, false, s);
@@ -602,21 +755,32 @@ haste_status_t haste_backward_dx_noalloc(haste_plan_t p, int32_t B, haste_dtype_
   a.band = t.band;
   a.n_bands = t.n_bands;
   a.n_chunks = t.n_chunks;
-  cudaError_t e = t.ns > 0 ? dx_v2(*p, B, W, dY, p->G, a.sh.L, a.dX_part, t, s)
+  cudaError_t e = t.ns > 0 ? dx_v2(*p, B, W, dY, false, a.dX_part, t, s)
                  : dt == HASTE_BF16  ? tail::launch_backward_dx<__nv_bfloat16>(a, false, s)
                                      : tail::launch_backward_dx<float>(a, false, s);
   if (e == cudaSuccess) e = tail::launch_dx_reduce(a.dX_part, dX, t.n_chunks, p->d, Bp, B, accumulate, s);
   return e == cudaSuccess ? HASTE_OK : cuda_fail(e, "haste_backward_dx_noalloc launch");
 }
 
-haste_status_t haste_bce_step(haste_plan_t p, int32_t B, haste_dtype_t dt, const void* X, const void* W,
-                              haste_targets_t pos, float grad_scale, float* loss, void* dW, float* dX,
-                              int accumulate, void* ws, size_t ws_bytes, haste_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// Optimizer update fused into the step kernel's dW readout (haste_bce_step_sgd).
+struct SgdUpdate {
+  float lr, momentum;
+  void* M;      // momentum [L, k] in W's dtype, NULL when momentum == 0
+  void* W_out;  // updated weights [L, k]
+};
+
+haste_status_t bce_step_impl(haste_plan_t p, int32_t B, haste_dtype_t dt, const void* X, const void* W,
+                             haste_targets_t pos, float grad_scale, float* loss, void* dW, const SgdUpdate* upd,
+                             float* dX, int accumulate, void* ws, size_t ws_bytes, haste_stream_t stream) {
   DeviceInfo di;
   haste_status_t st = device_info(di);
   if (st == HASTE_OK) st = check_tail(p, B, dt, di);
   if (st != HASTE_OK) return st;
-  if (!X || !W || !dW || !dX || !pos.row_ptr || !pos.ids) return fail(HASTE_ERR_INVALID_ARG, "NULL pointer");
+  if (!X || !W || (!upd && !dW) || !dX || !pos.row_ptr || !pos.ids) return fail(HASTE_ERR_INVALID_ARG, "NULL pointer");
   const int E = elem_bytes(dt);
   const int Bp = round_up(B, 128);
   if ((Bp / 128) * p->G + (E == 4 ? (p->G + 31) / 32 * 32 : p->G) > 512)
@@ -626,6 +790,10 @@ haste_status_t haste_bce_step(haste_plan_t p, int32_t B, haste_dtype_t dt, const
   const DxTiling t = dx_tiling(*p, Bp, E, di.sms, di.smem_optin);
   const TailWs w = tail_ws(*p, B, E, t);
   if ((st = check_ws(ws, ws_bytes, w.total)) != HASTE_OK) return st;
+  const bool v2p = use_v2(*p, Bp, E) && tail2::step_smem(Bp, p->k, p->G) <= (size_t)di.smem_optin && t.ns > 0;
+  if (upd && !v2p)
+    return fail(HASTE_ERR_UNSUPPORTED_SHAPE,
+                "the fused update needs bf16, G in {16,32,64}, k in {64,128} and B <= 256");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* wb = static_cast<uint8_t*>(ws);
   TailArgs a = make_args(*p, B);
@@ -641,7 +809,6 @@ haste_status_t haste_bce_step(haste_plan_t p, int32_t B, haste_dtype_t dt, const
   a.band = t.band;
   a.n_bands = t.n_bands;
   a.n_chunks = t.n_chunks;
-  const bool v2p = use_v2(*p, Bp, E) && tail2::step_smem(Bp, p->k, p->G) <= (size_t)di.smem_optin && t.ns > 0;
   const int grid = v2p ? (int)std::min<int64_t>(p->n_groups, di.sms)
                        : dt == HASTE_BF16 ? tail::step_grid<__nv_bfloat16>(a, di.sms) : tail::step_grid<float>(a, di.sms);
   if (grid <= 0 || grid > kMaxLossParts) return fail(HASTE_ERR_CUDA, "could not size the fused step grid");
@@ -663,7 +830,15 @@ haste_status_t haste_bce_step(haste_plan_t p, int32_t B, haste_dtype_t dt, const
       sa.pos_ptr = pos.row_ptr;
       sa.pos_ids = pos.ids;
       sa.grad_scale = grad_scale;
-      e = tail2::launch_step(p->G, p->k, sa, grid, a.Xt, W, s);
+      int mode = 0;
+      if (upd) {
+        sa.W_out = static_cast<__nv_bfloat16*>(upd->W_out);
+        sa.M = static_cast<__nv_bfloat16*>(upd->M);
+        sa.lr = upd->lr;
+        sa.momentum = upd->momentum;
+        mode = upd->momentum != 0.f ? 2 : 1;
+      }
+      e = tail2::launch_step(p->G, p->k, mode, sa, grid, a.Xt, W, s);
     } else {
       e = dt == HASTE_BF16 ? tail::launch_step<__nv_bfloat16>(a, grid, s) : tail::launch_step<float>(a, grid, s);
     }
@@ -671,9 +846,9 @@ haste_status_t haste_bce_step(haste_plan_t p, int32_t B, haste_dtype_t dt, const
   if (e == cudaSuccess) {
     ProfScope ps("tail_dx", s);
     if (v2p)
-      e = dx_v2(*p, B, W, a.dY_out, (int64_t)Bp * p->G, p->G, a.dX_part, t, s);
+      e = dx_v2(*p, B, W, a.dY_out, true, a.dX_part, t, s);
     else if (t.ns > 0)
-      e = dx_v2(*p, B, W, a.dY_out, p->G, a.sh.L, a.dX_part, t, s);
+      e = dx_v2(*p, B, W, a.dY_out, false, a.dX_part, t, s);
     else
       e = dt == HASTE_BF16 ? tail::launch_backward_dx<__nv_bfloat16>(a, true, s)
                            : tail::launch_backward_dx<float>(a, true, s);
@@ -683,7 +858,30 @@ haste_status_t haste_bce_step(haste_plan_t p, int32_t B, haste_dtype_t dt, const
     e = tail::launch_dx_reduce(a.dX_part, dX, t.n_chunks, p->d, Bp, B, accumulate, s, loss ? a.loss_part : nullptr,
                                grid, grad_scale, loss);
   }
-  return e == cudaSuccess ? HASTE_OK : cuda_fail(e, "haste_bce_step launch");
+  return e == cudaSuccess ? HASTE_OK : cuda_fail(e, upd ? "haste_bce_step_sgd launch" : "haste_bce_step launch");
+}
+
+}  // namespace
+
+extern "C" {
+
+haste_status_t haste_bce_step(haste_plan_t p, int32_t B, haste_dtype_t dt, const void* X, const void* W,
+                              haste_targets_t pos, float grad_scale, float* loss, void* dW, float* dX,
+                              int accumulate, void* ws, size_t ws_bytes, haste_stream_t stream) {
+  return bce_step_impl(p, B, dt, X, W, pos, grad_scale, loss, dW, nullptr, dX, accumulate, ws, ws_bytes, stream);
+}
+
+haste_status_t haste_bce_step_sgd(haste_plan_t p, int32_t B, haste_dtype_t dt, const void* X, const void* W,
+                                  haste_targets_t pos, float grad_scale, float* loss, float lr, float momentum,
+                                  void* M, void* W_out, float* dX, int accumulate, void* ws, size_t ws_bytes,
+                                  haste_stream_t stream) {
+  if (!W_out) return fail(HASTE_ERR_INVALID_ARG, "W_out is NULL");
+  if (W_out == W) return fail(HASTE_ERR_INVALID_ARG, "W_out must not be W: the dX pass reads W after the update");
+  if (momentum != 0.f && !M) return fail(HASTE_ERR_INVALID_ARG, "momentum != 0 needs the momentum buffer M");
+  if (M && (M == W || M == W_out)) return fail(HASTE_ERR_INVALID_ARG, "M must be its own buffer");
+  if (!(lr == lr) || !(momentum == momentum)) return fail(HASTE_ERR_INVALID_ARG, "lr and momentum must be numbers");
+  const SgdUpdate u{lr, momentum, momentum != 0.f ? M : nullptr, W_out};
+  return bce_step_impl(p, B, dt, X, W, pos, grad_scale, loss, nullptr, &u, dX, accumulate, ws, ws_bytes, stream);
 }
 
 // ------------------------------------------------------------------- head
@@ -721,7 +919,7 @@ static size_t topk_ws(const haste_plan_s& p, int B, int E, int n_buckets, int kp
 }
 
 size_t haste_topk_workspace_size(haste_plan_t p, int32_t B, haste_dtype_t dt, int32_t n_buckets, int32_t kp) {
-  if (!p || B <= 0 || n_buckets <= 0 || kp <= 0) return 0;
+  if (!p || B <= 0 || n_buckets <= 0 || kp <= 0 || check_plan_device(p) != HASTE_OK) return 0;
   size_t cand;
   return topk_ws(*p, B, elem_bytes(dt), n_buckets, kp, &cand);
 }

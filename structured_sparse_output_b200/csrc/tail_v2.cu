@@ -9,10 +9,14 @@
 //   warp 4     MMA issuer (one thread): issues each group's forward and dW
 //              product as soon as its inputs are ready, so the tensor core works
 //              while the epilogue runs;
-//   warps 5-12 epilogue: logits leave TMEM only as the BCE gradient (bf16, to
+//   warps 5-20 epilogue: logits leave TMEM only as the BCE gradient (bf16, to
 //              shared memory for the dW product and to the group-major gradient
 //              buffer of the dX pass); the BCE of group i+1 comes before the dW
-//              readout of group i, so the dW product runs behind it.
+//              readout of group i, so the dW product runs behind it.  The readout
+//              writes dW, or (kUpd > 0) applies an SGD update to the group's
+//              weights while dW is on chip: M' = momentum * M + dW (kUpd = 2) or
+//              M' = dW (kUpd = 1), W' = W - lr * M', with W' written to a
+//              separate buffer (the dX pass still reads W) and M' over M.
 //
 // The dX pass that reads the gradient buffer is in dx_band.cu.
 
@@ -24,7 +28,10 @@ namespace v2 {
 struct StepArgs {
   TailShape sh;
   const int32_t* idx;
-  __nv_bfloat16* dW;
+  __nv_bfloat16* dW;      // kUpd = 0
+  __nv_bfloat16* W_out;   // kUpd > 0: updated weights [L, k]
+  __nv_bfloat16* M;       // kUpd = 2: momentum [L, k], updated in place
+  float lr, momentum;
   __nv_bfloat16* dY_out;  // group-major gradient buffer [n_groups, Bp, G]
   float* loss_part;
   const int32_t* pos_ptr;
@@ -57,7 +64,7 @@ __device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
 // Bounded wait; on timeout the CTA-wide abort flag is raised.
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
   if (*abort_flag) return false;
-  if (!mbar_wait(bar, parity)) {
+  if (!mbar_wait(bar, parity, g_wait_limit_ns)) {
     *abort_flag = 1;
     return false;
   }
@@ -75,10 +82,11 @@ __device__ __forceinline__ void publish_all(uint64_t* full_bar) {
 // ============================================================ k_step2
 constexpr int kStepProd = 4;       // producer warps: two per ring stage
 constexpr int kStepMma = kStepProd;  // warp id of the MMA issuer
-constexpr int kStepThreads = 32 * (kStepProd + 1 + 8);  // producers, MMA warp, 8 epilogue warps
+constexpr int kStepEpi = 16;       // epilogue warps: 4 lane quarters x 2 column halves x 2 batch tiles
+constexpr int kStepThreads = 32 * (kStepProd + 1 + kStepEpi);  // producers, MMA warp, epilogue warps
 constexpr int kMaxPosReg = 8;      // positives per batch row kept in registers
 
-template <int kG, int kK>
+template <int kG, int kK, int kUpd>
 __global__ void __launch_bounds__(kStepThreads, 1)
     k_step2(StepArgs a, const __nv_bfloat16* __restrict__ Xt, const __nv_bfloat16* __restrict__ W) {
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -97,9 +105,10 @@ __global__ void __launch_bounds__(kStepThreads, 1)
   uint64_t* dy_full = bars + 6;      // [2] dY in shared memory
   uint64_t* dw_full = bars + 8;      // [2] dW in TMEM
   uint64_t* tmem_empty = bars + 10;  // [2] dW accumulator D read out
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 12);
+  uint64_t* done = bars + 12;        // every MMA of the CTA finished
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 13);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
-  float* red = reinterpret_cast<float*>(tslot + 2);  // 8 warp partials
+  float* red = reinterpret_cast<float*>(tslot + 2);  // kStepEpi warp partials
 
   const int w = warp_id(), lane = lane_id();
   if (threadIdx.x == 0) {
@@ -107,10 +116,11 @@ __global__ void __launch_bounds__(kStepThreads, 1)
       mbar_init(&full[s], 32 * kStepProd / 2);
       mbar_init(&empty[s], 1);
       mbar_init(&fwd_full[s], 1);
-      mbar_init(&dy_full[s], 8);
+      mbar_init(&dy_full[s], kStepEpi);
       mbar_init(&dw_full[s], 1);
-      mbar_init(&tmem_empty[s], 8);
+      mbar_init(&tmem_empty[s], kStepEpi);
     }
+    mbar_init(done, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -193,11 +203,12 @@ __global__ void __launch_bounds__(kStepThreads, 1)
     // which holds once dW(j-2) was issued (its BCE had finished reading F);
     // dW(j) needs the BCE of j (dy_full) and D(j&1) read out for j-2
     // (tmem_empty).  Lane 0 polls; the decisions are broadcast so the warp stays
-    // converged.  No progress for kWaitLimitNs raises the abort flag.
+    // converged.  No progress for the wait limit raises the abort flag.
     const uint32_t idesc_f = make_idesc(1, 1, 0, 128, kG);
     const uint32_t idesc_w = make_idesc(1, 0, 1, 128, kG);
     int nf = 0, nd = 0;
     uint64_t t_last = globaltimer_ns();
+    const uint64_t limit = g_wait_limit_ns;
     while (nd < n_items) {
       if (*abort_flag) break;
       bool did = false;
@@ -250,7 +261,7 @@ __global__ void __launch_bounds__(kStepThreads, 1)
       if (did) {
         t_last = globaltimer_ns();
       } else {
-        if (globaltimer_ns() - t_last > kWaitLimitNs) {
+        if (globaltimer_ns() - t_last > limit) {
           if (lane == 0) {
             *abort_flag = 1;
             record_error(kErrTimeout);
@@ -261,57 +272,60 @@ __global__ void __launch_bounds__(kStepThreads, 1)
         __nanosleep(32);
       }
     }
+    // Also after an abort: the CTA frees TMEM and exits only once every MMA it
+    // issued has finished writing TMEM and reading shared memory.
+    if (lane == 0) mma_commit(done);
+    __syncwarp();
+    (void)__all_sync(0xffffffffu, mbar_wait(done, 0));
   } else {
     // ------------------------------------------------------------- epilogue
-    // warp (q, hh): TMEM lane quarter q, label columns [hh*CH, hh*CH + CH)
-    const int ew = w - kStepMma - 1, q = w & 3, hh = ew >> 2;
+    // warp (q, hh, tt): TMEM lane quarter q.  BCE: batch tile tt, label columns
+    // [hh*CH, hh*CH + CH) (warps of a tile beyond the batch only take part in the
+    // barriers).  dW readout: slots 32q.., label columns [hh*CH + tt*RC, +RC).
+    constexpr int RC = CH / 2;
+    const int ew = w - kStepMma - 1, q = w & 3, hh = (ew >> 2) & 1, tt = ew >> 3;
     const int r = q * 32 + lane;  // row inside a 128-row tile (and dW slot)
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     const float scale = a.grad_scale;
+    const bool has_tile = tt < n_bt;
+    const int b = tt * 128 + r;
+    const bool live = has_tile && b < sh.B;
     float loss_acc = 0.f;
-    // this thread's positives (tail-local ids), one batch row per 128-row tile
-    int pos[2][kMaxPosReg];
-    int npos[2] = {0, 0}, pbeg[2] = {0, 0};
-#pragma unroll
-    for (int t = 0; t < 2; ++t) {
-      const int b = t * 128 + r;
-      if (t < n_bt && b < sh.B) {
-        pbeg[t] = a.pos_ptr[b];
-        npos[t] = a.pos_ptr[b + 1] - pbeg[t];
-      }
-#pragma unroll
-      for (int e = 0; e < kMaxPosReg; ++e) pos[t][e] = e < npos[t] ? a.pos_ids[pbeg[t] + e] : -1;
+    // this thread's positives (tail-local ids)
+    int pos[kMaxPosReg];
+    int npos = 0, pbeg = 0;
+    if (live) {
+      pbeg = a.pos_ptr[b];
+      npos = a.pos_ptr[b + 1] - pbeg;
     }
+#pragma unroll
+    for (int e = 0; e < kMaxPosReg; ++e) pos[e] = e < npos ? a.pos_ids[pbeg + e] : -1;
     auto bce = [&](int i) -> bool {
       const int64_t g = gb + i;
       const int s = i & 1;
       if (!wait_or_abort(&fwd_full[s], (i >> 1) & 1, abort_flag)) return false;
       tc_fence_after();
-      const int64_t l0 = g * kG + hh * CH;  // first label of this warp's columns
-      uint8_t* dyrow = gbase + DY(s);
-      __nv_bfloat16* dyg = a.dY_out + g * (int64_t)Bp * kG;
-#pragma unroll
-      for (int t = 0; t < 2; ++t) {
-        if (t >= n_bt) break;
-        const int b = t * 128 + r;
-        const bool live = b < sh.B;
+      if (has_tile) {
+        const int64_t l0 = g * kG + hh * CH;  // first label of this warp's columns
+        uint8_t* dyrow = gbase + DY(s);
+        __nv_bfloat16* dyg = a.dY_out + g * (int64_t)Bp * kG;
         const float sl = live ? scale : 0.f, hs = 0.5f * sl;  // rows beyond B get dY = 0
         uint32_t ym = 0;
 #pragma unroll
         for (int e = 0; e < kMaxPosReg; ++e) {
-          const int64_t l = (int64_t)pos[t][e] - l0;
-          if (pos[t][e] >= 0 && l >= 0 && l < CH) ym |= 1u << l;
+          const int64_t l = (int64_t)pos[e] - l0;
+          if (pos[e] >= 0 && l >= 0 && l < CH) ym |= 1u << l;
         }
-        for (int e = kMaxPosReg; e < npos[t]; ++e) {  // rows with many positives
-          const int64_t l = (int64_t)a.pos_ids[pbeg[t] + e] - l0;
+        for (int e = kMaxPosReg; e < npos; ++e) {  // rows with many positives
+          const int64_t l = (int64_t)a.pos_ids[pbeg + e] - l0;
           if (l >= 0 && l < CH) ym |= 1u << l;
         }
 #pragma unroll
         for (int c = 0; c < CH; c += 16) {
           constexpr int NC = CH < 16 ? CH : 16;
           float z[16];
-          if constexpr (NC == 8) tmem_ld8(F(s) + lane_off + (uint32_t)(t * kG + hh * CH + c), z);
-          else tmem_ld16(F(s) + lane_off + (uint32_t)(t * kG + hh * CH + c), z);
+          if constexpr (NC == 8) tmem_ld8(F(s) + lane_off + (uint32_t)(tt * kG + hh * CH + c), z);
+          else tmem_ld16(F(s) + lane_off + (uint32_t)(tt * kG + hh * CH + c), z);
           tmem_wait_ld();
           // y = 0 everywhere first (positives are rare), then the few positive
           // columns are corrected: dY -= scale, loss -= z.
@@ -358,18 +372,31 @@ __global__ void __launch_bounds__(kStepThreads, 1)
       const int s = i & 1;
       if (!wait_or_abort(&dw_full[s], (i >> 1) & 1, abort_flag)) return false;
       tc_fence_after();
-      // dW readout: row = slot r, columns = this warp's labels
+      // dW readout: row = slot r, columns = this warp's RC labels
+      const int c0 = hh * CH + tt * RC;
+      float v[16];
+      if constexpr (RC == 16) tmem_ld16(D(s) + lane_off + (uint32_t)c0, v);
+      else if constexpr (RC == 8) tmem_ld8(D(s) + lane_off + (uint32_t)c0, v);
+      else tmem_ld4(D(s) + lane_off + (uint32_t)c0, v);
+      tmem_wait_ld();
+      if (r < kK) {
+        const int64_t off0 = (g * kG + c0) * kK + r;  // (label, slot r); lanes: consecutive slots
+        if constexpr (kUpd == 0) {
 #pragma unroll
-      for (int c = 0; c < CH; c += 16) {
-        constexpr int NC = CH < 16 ? CH : 16;
-        float v[16];
-        if constexpr (NC == 8) tmem_ld8(D(s) + lane_off + (uint32_t)(hh * CH + c), v);
-        else tmem_ld16(D(s) + lane_off + (uint32_t)(hh * CH + c), v);
-        tmem_wait_ld();
-        if (r < kK) {
-          __nv_bfloat16* dst = a.dW + (g * kG + hh * CH + c) * kK + r;
+          for (int e = 0; e < RC; ++e) a.dW[off0 + (int64_t)e * kK] = __float2bfloat16_rn(v[e]);
+        } else {
+          float wv[RC], mv[RC];
 #pragma unroll
-          for (int e = 0; e < NC; ++e) dst[(int64_t)e * kK] = __float2bfloat16_rn(v[e]);
+          for (int e = 0; e < RC; ++e) {
+            wv[e] = __bfloat162float(W[off0 + (int64_t)e * kK]);
+            mv[e] = kUpd == 2 ? __bfloat162float(a.M[off0 + (int64_t)e * kK]) : 0.f;
+          }
+#pragma unroll
+          for (int e = 0; e < RC; ++e) {
+            const float m = kUpd == 2 ? fmaf(a.momentum, mv[e], v[e]) : v[e];
+            if constexpr (kUpd == 2) a.M[off0 + (int64_t)e * kK] = __float2bfloat16_rn(m);
+            a.W_out[off0 + (int64_t)e * kK] = __float2bfloat16_rn(fmaf(-a.lr, m, wv[e]));
+          }
         }
       }
       tc_fence_before();
@@ -382,15 +409,15 @@ __global__ void __launch_bounds__(kStepThreads, 1)
       if (i + 1 < n_items && !bce(i + 1)) break;
       if (!readout(i)) break;
     }
-    // deterministic loss reduction over the 8 epilogue warps (named barrier 1)
+    // deterministic loss reduction over the epilogue warps (named barrier 1)
     float v = loss_acc;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     if (lane == 0) red[ew] = v;
-    named_bar(1, 256);
+    named_bar(1, 32 * kStepEpi);
     if (ew == 0 && lane == 0) {
       float t = 0.f;
-      for (int j = 0; j < 8; ++j) t += red[j];
+      for (int j = 0; j < kStepEpi; ++j) t += red[j];
       a.loss_part[blockIdx.x] = t;
     }
   }
@@ -412,10 +439,10 @@ bool supported(int G, int k, int Bp) {
 }
 
 size_t step_smem(int Bp, int k, int G) { return v2::step_layout(Bp, k, G).total; }
-template <int kG, int kK>
+template <int kG, int kK, int kUpd>
 cudaError_t launch_step_t(const v2::StepArgs& a, int grid, const void* Xt, const void* W, cudaStream_t st) {
   const size_t smem = step_smem(a.sh.Bp, kK, kG);
-  auto kern = v2::k_step2<kG, kK>;
+  auto kern = v2::k_step2<kG, kK, kUpd>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   kern<<<grid, v2::kStepThreads, smem, st>>>(a, static_cast<const __nv_bfloat16*>(Xt),
@@ -472,9 +499,28 @@ cudaError_t tmap_2d(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t 
     default: return cudaErrorInvalidValue;                             \
   }
 
-cudaError_t launch_step(int G, int k, const v2::StepArgs& a, int grid, const void* Xt, const void* W,
+template <int kG, int kK>
+cudaError_t launch_step_dw(const v2::StepArgs& a, int grid, const void* Xt, const void* W, cudaStream_t st) {
+  return launch_step_t<kG, kK, 0>(a, grid, Xt, W, st);
+}
+template <int kG, int kK>
+cudaError_t launch_step_sgd(const v2::StepArgs& a, int grid, const void* Xt, const void* W, cudaStream_t st) {
+  return launch_step_t<kG, kK, 1>(a, grid, Xt, W, st);
+}
+template <int kG, int kK>
+cudaError_t launch_step_sgdm(const v2::StepArgs& a, int grid, const void* Xt, const void* W, cudaStream_t st) {
+  return launch_step_t<kG, kK, 2>(a, grid, Xt, W, st);
+}
+
+// upd: 0 writes dW; 1 applies SGD (W' = W - lr dW); 2 SGD with momentum.
+cudaError_t launch_step(int G, int k, int upd, const v2::StepArgs& a, int grid, const void* Xt, const void* W,
                         cudaStream_t st) {
-  HASTE_V2_DISPATCH(launch_step_t, a, grid, Xt, W, st)
+  if (upd == 1) {
+    HASTE_V2_DISPATCH(launch_step_sgd, a, grid, Xt, W, st)
+  } else if (upd == 2) {
+    HASTE_V2_DISPATCH(launch_step_sgdm, a, grid, Xt, W, st)
+  }
+  HASTE_V2_DISPATCH(launch_step_dw, a, grid, Xt, W, st)
 }
 
 }  // namespace tail2

@@ -80,7 +80,7 @@ __device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
 
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
   if (*abort_flag) return false;
-  if (!mbar_wait(bar, parity)) {
+  if (!mbar_wait(bar, parity, g_wait_limit_ns)) {
     *abort_flag = 1;
     return false;
   }
@@ -103,7 +103,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* empty = bars + 2;     // [2] stage consumed by the forward product
   uint64_t* fwd_full = bars + 4;  // [2] logits in TMEM
   uint64_t* f_empty = bars + 6;   // [2] logits read out (count: 8 epilogue warps)
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 8);
+  uint64_t* done = bars + 8;      // every MMA of the CTA finished
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 9);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
 
   const int w = warp_id(), lane = lane_id();
@@ -114,6 +115,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&fwd_full[s], 1);
       mbar_init(&f_empty[s], 8);
     }
+    mbar_init(done, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -197,6 +199,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
     }
+    // also after an abort: TMEM is freed only once every issued MMA has finished
+    if (lane == 0) mma_commit(done);
+    __syncwarp();
+    (void)__all_sync(0xffffffffu, mbar_wait(done, 0));
   } else {
     // ------------------------------------------------------------- epilogue
     // warp (q, hh): TMEM lane quarter q, label columns [hh*CH, hh*CH + CH)

@@ -76,3 +76,54 @@ def test_binding_rejects_host_tensors():
     with pytest.raises(ValueError, match="CUDA tensors"):
         H._tptr(torch.zeros(8))
     assert H._tptr(None) is None
+
+
+def _fake_plan(device=0):
+    """Shape fields of a plan without a library handle (no GPU needed): 4 groups of
+    G = 16 labels, k = 64, d = 128, on CUDA device `device`."""
+    return H.Plan(None, 4, 16, 64, 128, device)
+
+
+def test_binding_checks_shapes_dtypes_and_devices_before_any_pointer():
+    """Wrong shapes, dtypes or devices never reach the library: every case raises
+    ValueError in the binding (these run without a GPU and without a plan handle)."""
+    torch = pytest.importorskip("torch")
+    bf, f32, i32 = torch.bfloat16, torch.float32, torch.int32
+    p = _fake_plan()
+    B, L, k, d = 8, 64, 64, 128
+    X, W = torch.zeros(B, d, dtype=bf), torch.zeros(L, k, dtype=bf)
+    cases = [
+        (lambda: H.haste_forward(p, X, torch.zeros(L, k + 1, dtype=bf), torch.zeros(B, L, dtype=bf), None), "shape"),
+        (lambda: H.haste_forward(p, torch.zeros(B, d + 8, dtype=bf), W, torch.zeros(B, L, dtype=bf), None), "shape"),
+        (lambda: H.haste_forward(p, X, W, torch.zeros(B, L, dtype=f32), None), "dtype"),
+        (lambda: H.haste_backward_dw(p, X, torch.zeros(B, L + 16, dtype=bf), torch.zeros(L, k, dtype=bf), None),
+         "shape"),
+        (lambda: H.haste_backward_dx(p, W, torch.zeros(B, L, dtype=f32), torch.zeros(B, d), None), "dtype"),
+        (lambda: H.haste_backward_dx(p, W, torch.zeros(B, L, dtype=bf), torch.zeros(B, d, dtype=bf), None), "dtype"),
+        (lambda: H.haste_backward_dx_noalloc(p, W, torch.zeros(B, L, dtype=bf), torch.zeros(B, d + 1)), "shape"),
+        (lambda: H.haste_bce_step(p, X, W, torch.zeros(B, dtype=i32), torch.zeros(3, dtype=i32), 0.1, None,
+                                  torch.zeros(L, k, dtype=bf), torch.zeros(B, d), None), "row_ptr"),
+        (lambda: H.haste_bce_step(p, X, W, torch.zeros(B + 1, dtype=i32), torch.zeros(3, dtype=torch.int64), 0.1,
+                                  None, torch.zeros(L, k, dtype=bf), torch.zeros(B, d), None), "ids"),
+        (lambda: H.haste_topk(p, X, W, 5, 4, 2, torch.zeros(B, 4), torch.zeros(B, 5, dtype=i32), None), "shape"),
+        (lambda: H.haste_head_forward(X, torch.zeros(16, d + 8, dtype=bf), torch.zeros(B, 16, dtype=bf), None),
+         "shape"),
+        (lambda: H.haste_head_backward(X, torch.zeros(16, d, dtype=bf), torch.zeros(B, 16, dtype=bf),
+                                       torch.zeros(16, d, dtype=bf), torch.zeros(B, d, dtype=bf), None), "dtype"),
+        # right shapes, host tensors
+        (lambda: H.haste_forward(p, X, W, torch.zeros(B, L, dtype=bf), None), "CUDA"),
+        (lambda: H.haste_head_backward(X, torch.zeros(16, d, dtype=bf), torch.zeros(B, 16, dtype=bf),
+                                       torch.zeros(16, d, dtype=bf), torch.zeros(B, d), None), "CUDA"),
+    ]
+    for i, (call, what) in enumerate(cases):
+        with pytest.raises(ValueError, match=what):
+            call()
+
+
+def test_binding_refuses_tensors_off_the_plans_device():
+    """A plan lives on one device: tensors elsewhere are refused by name."""
+    torch = pytest.importorskip("torch")
+    p = _fake_plan(device=1)
+    X, W = torch.zeros(8, 128, dtype=torch.bfloat16), torch.zeros(64, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="X is on cpu"):
+        H.haste_forward(p, X, W, torch.zeros(8, 64, dtype=torch.bfloat16), None)

@@ -52,6 +52,14 @@ def _run(run):
     assert H.haste_device_status() == H.HASTE_OK
 
 
+def _row_subset(pos, rows):
+    """The positives CSR of the given batch rows only."""
+    rp, ids = pos
+    sub_rp = np.concatenate([[0], np.cumsum([rp[b + 1] - rp[b] for b in rows])]).astype(np.int32)
+    sub_ids = np.concatenate([ids[rp[b]:rp[b + 1]] for b in rows]).astype(np.int32)
+    return sub_rp, sub_ids
+
+
 @pytest.mark.parametrize("name", ["670k", "3m", "8.6m"])
 def test_fused_step_full_size_sampled(name):
     import bench
@@ -65,20 +73,28 @@ def test_fused_step_full_size_sampled(name):
     # bitwise run-to-run determinism of every output of the step
     for a, b in ((dW1, run.dW), (dX1, run.dX), (dWh1, run.dWh), (dXh1, run.dXh), (loss1, run.loss)):
         assert _same(a, b)
-    ls, ss, bs, fs = _samples(wl)
     scale = 1.0 / wl.B
+    # the tail loss over every sample and label
+    r_loss = O.bce_loss(inp.X, inp.W, inp.idx, wl.G, inp.tail_pos[0], inp.tail_pos[1], scale)
+    assert abs(float(run.loss[0].item()) - r_loss) <= 5e-3 * abs(r_loss), (float(run.loss[0].item()), r_loss)
+    ls, ss, bs, fs = _samples(wl, n_dw=400, n_dx=64)
     dW = run.dW.float().cpu().numpy()
     dX = run.dX.cpu().numpy()
     r_dw = O.dw_at(inp.X, inp.W, inp.idx, wl.G, ls, ss, pos=inp.tail_pos, scale=scale)
     r_dx = O.dx_at(inp.X, inp.W, inp.idx, wl.G, bs, fs, pos=inp.tail_pos, scale=scale)
     assert_close(dW[ls, ss].astype(np.float64), r_dw, f"{name} dW samples")
     assert_close(dX[bs, fs].astype(np.float64), r_dx, f"{name} dX samples")
+    if name == "670k":
+        # whole dX rows: a row's gradient depends on that row only, so the oracle's
+        # step over a subset of rows (same scale) gives those rows exactly
+        rows = np.array([0, 1, 2, 3, 128, wl.B - 1])
+        _, _, _, r_rows = O.bce_step(inp.X[rows], inp.W, inp.idx, wl.G, *_row_subset(inp.tail_pos, rows), scale)
+        assert_close(dX[rows].astype(np.float64), r_rows, f"{name} dX rows {rows.tolist()}")
     # the dense head in full
     h_loss, _, h_dWh, h_dXh = O.head_step(inp.Xh, inp.Wh, inp.head_pos[0], inp.head_pos[1], scale)
     assert_close(to_np64(run.dWh), h_dWh, f"{name} head dWh")
     assert_close(to_np64(run.dXh), h_dXh, f"{name} head dXh")
     assert abs(float(run.loss[1].item()) - h_loss) <= 5e-3 * abs(h_loss)
-    assert np.isfinite(float(run.loss[0].item())) and float(run.loss[0].item()) > 0.0
 
 
 @pytest.mark.parametrize("name", ["sweep16", "sweep32", "sweep64"])

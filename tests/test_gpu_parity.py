@@ -58,6 +58,9 @@ TAIL_CASES = [
     dict(B=100, d=200, n_groups=150, G=16, k=64, dtype="bf16"),
     # fewer groups than group chunks: one group per CTA, one batch tile
     dict(B=64, d=768, n_groups=5, G=32, k=128, dtype="bf16"),
+    # three batch tiles (k = 64: padded M = 128 dW product), and a ragged third tile of one row
+    dict(B=384, d=768, n_groups=300, G=64, k=64, dtype="bf16"),
+    dict(B=257, d=1024, n_groups=129, G=32, k=128, dtype="bf16"),
     # four bands, the last one 232 features wide
     dict(B=256, d=1000, n_groups=97, G=16, k=128, dtype="bf16"),
     # degenerate counts: a batch of one row; a single group (one chunk, one CTA per band)
@@ -247,3 +250,180 @@ def test_bounded_wait_timeout_is_reported_and_context_survives():
     assert H.haste_device_status() == H.HASTE_OK          # cleared after reporting
     a = torch.ones(1024, device="cuda")
     assert float((a * 2).sum().item()) == 2048.0
+
+
+def test_short_wait_limit_reaches_the_abort_paths_and_the_context_survives():
+    """A 1 ns limit on the pipelined kernels' inter-warp waits makes the first wait
+    of the step kernel, the dX band kernel and the top-k kernel run out, so each
+    takes its abort path (raise the CTA's abort flag, drain its own copies, commit
+    and wait for its issued MMAs, free TMEM).  The timeout is reported once; with
+    the default limit restored, the same calls give the oracle's results."""
+    c = dict(B=256, d=768, n_groups=300, G=32, k=128, dtype="bf16", H=0, p=5)
+    idx, X, W, tpos, _ = _step_inputs(c)
+    plan = H.haste_plan(idx, c["G"], c["d"])
+    scale = 1.0 / c["B"]
+    nb, K, kp = 37, 5, 4
+    ws = torch.empty(H.haste_topk_workspace_size(plan, c["B"], H.HASTE_BF16, nb, kp), dtype=torch.uint8,
+                     device="cuda")
+    ov = torch.empty((c["B"], K), device="cuda")
+    oi = torch.empty((c["B"], K), dtype=torch.int32, device="cuda")
+    try:
+        H.haste_set_wait_limit_ns(1)
+        _run_step(plan, X, W, tpos, scale)
+        assert H.haste_device_status() == H.HASTE_ERR_TIMEOUT
+        H.haste_topk(plan, to_torch(X), to_torch(W), K, kp, nb, ov, oi, ws)
+        assert H.haste_device_status() == H.HASTE_ERR_TIMEOUT
+    finally:
+        H.haste_set_wait_limit_ns(0)
+    assert H.haste_device_status() == H.HASTE_OK
+    loss, dW, dX = _run_step(plan, X, W, tpos, scale)
+    assert H.haste_device_status() == H.HASTE_OK
+    r_loss, _, r_dW, r_dX = O.bce_step(X, W, idx, c["G"], tpos[0], tpos[1], scale)
+    assert abs(float(loss.item()) - r_loss) <= 5e-3 * abs(r_loss)
+    assert_close(to_np64(dW), r_dW, "dW after the aborted call")
+    assert_close(to_np64(dX), r_dX, "dX after the aborted call")
+    with pytest.raises(H.HasteError):
+        H.haste_set_wait_limit_ns(10 ** 12)       # above the 2 s default
+
+
+SGD_CASES = [
+    dict(B=256, d=768, n_groups=300, G=64, k=128, dtype="bf16", H=0, p=8, lr=4.0, mu=0.9),
+    dict(B=130, d=384, n_groups=250, G=32, k=64, dtype="bf16", H=0, p=5, lr=2.0, mu=0.0),
+    dict(B=100, d=256, n_groups=120, G=16, k=64, dtype="bf16", H=0, p=5, lr=3.0, mu=0.5),
+]
+
+
+@pytest.mark.parametrize("case", SGD_CASES, ids=lambda c: _case_id(c) + f"_mu{c['mu']}")
+def test_fused_step_with_sgd_update_two_steps(case):
+    """haste_bce_step_sgd over two steps, alternating two weight buffers as a
+    training loop does: the loss and dX of each step use that step's input
+    weights, the momentum buffer and the new weights follow the oracle's SGD
+    update.  lr is large so that the update, not the bf16 rounding of W', decides
+    the comparison of W' - W."""
+    idx, X, W0, tpos, _ = _step_inputs(case)
+    B, d, G, k = case["B"], case["d"], case["G"], case["k"]
+    lr, mu = case["lr"], case["mu"]
+    plan = H.haste_plan(idx, G, d)
+    scale = 1.0 / B
+    M0 = I.make_normal((plan.L, k), 0.03, 0, 4, "bf16") if mu else None
+    Xt = to_torch(X)
+    rp, ids = to_torch(tpos[0]), to_torch(tpos[1])
+    ws = _ws(plan, B, H.HASTE_BF16)
+    bufs = [to_torch(W0), torch.empty_like(to_torch(W0))]
+    Mt = to_torch(M0) if mu else None
+    W_ref, M_ref = W0, M0
+    for step in range(2):
+        Win, Wout = bufs[step % 2], bufs[(step + 1) % 2]
+        Win_before = Win.clone()
+        loss = torch.zeros(1, device="cuda")
+        dX = torch.full((B, d), float("nan"), device="cuda")
+        H.haste_bce_step_sgd(plan, Xt, Win, rp, ids, scale, loss, lr, mu, Mt, Wout, dX, ws)
+        torch.cuda.synchronize()
+        assert H.haste_device_status() == H.HASTE_OK
+        assert torch.equal(Win.view(torch.int16), Win_before.view(torch.int16))   # W is only read
+        r_loss, r_dX, r_W, r_M = O.bce_step_sgd(X, W_ref, M_ref, idx, G, tpos[0], tpos[1], scale, lr, mu)
+        assert abs(float(loss.item()) - r_loss) <= 5e-3 * abs(r_loss), (step, float(loss.item()), r_loss)
+        assert_close(to_np64(dX), r_dX, f"dX, step {step + 1}")
+        W_in64 = O.to_f64(W_ref)
+        assert_close(to_np64(Wout) - W_in64, r_W - W_in64, f"W' - W, step {step + 1}")
+        if mu:
+            assert_close(to_np64(Mt), r_M, f"momentum, step {step + 1}")
+            M_ref = Mt.view(torch.int16).cpu().numpy().view(np.uint16).copy()
+        # the next step starts from the GPU's rounded weights, as the oracle's input
+        W_ref = Wout.view(torch.int16).cpu().numpy().view(np.uint16).copy()
+
+
+def test_fused_update_argument_errors():
+    idx = I.make_idx(40, 64, 256, 0)
+    plan = H.haste_plan(idx, 32, 256)
+    B = 8
+    X = torch.zeros((B, 256), dtype=torch.bfloat16, device="cuda")
+    W = torch.zeros((40 * 32, 64), dtype=torch.bfloat16, device="cuda")
+    rp = torch.zeros(B + 1, dtype=torch.int32, device="cuda")
+    ids = torch.zeros(1, dtype=torch.int32, device="cuda")
+    dX = torch.empty((B, 256), device="cuda")
+    ws = _ws(plan, B, H.HASTE_BF16)
+    with pytest.raises(H.HasteError) as e:                       # the update must not overwrite W
+        H.haste_bce_step_sgd(plan, X, W, rp, ids, 0.1, None, 0.1, 0.0, None, W, dX, ws)
+    assert e.value.status == H.HASTE_ERR_INVALID_ARG
+    with pytest.raises(ValueError):                             # momentum needs its buffer
+        H.haste_bce_step_sgd(plan, X, W, rp, ids, 0.1, None, 0.1, 0.9, None, torch.empty_like(W), dX, ws)
+    Xf = torch.zeros((B, 256), device="cuda")
+    with pytest.raises(H.HasteError) as e:                       # fp32 runs the staged kernels: no fused update
+        H.haste_bce_step_sgd(plan, Xf, W.float(), rp, ids, 0.1, None, 0.1, 0.0, None, torch.empty_like(W.float()),
+                             dX, _ws(plan, B, H.HASTE_F32))
+    assert e.value.status == H.HASTE_ERR_UNSUPPORTED_SHAPE
+
+
+def _rewire(idx, d, frac_groups, frac_slots, seed):
+    """A random prune/regrow edit, the test's own rule: in a fraction of the groups,
+    drop a fraction of the features and draw replacements among the features the
+    group does not use, then sort the row.  Returns (groups, rows, new idx)."""
+    rng = np.random.default_rng(seed)
+    n_groups, k = idx.shape
+    groups = np.sort(rng.choice(n_groups, max(1, int(frac_groups * n_groups)), replace=False)).astype(np.int32)
+    rows = idx[groups].copy()
+    n_drop = max(1, int(frac_slots * k))
+    for r in range(len(groups)):
+        kept = rows[r][rng.choice(k, k - n_drop, replace=False)]
+        new = rng.choice(np.setdiff1d(np.arange(d), rows[r]), n_drop, replace=False)
+        rows[r] = np.sort(np.concatenate([kept, new]))
+    out = idx.copy()
+    out[groups] = rows
+    return groups, rows, out
+
+
+@pytest.mark.parametrize("n_groups,k,d", [(20_944, 128, 768), (1000, 64, 97), (7, 5, 5), (134_376, 128, 768)])
+def test_plan_update_is_bit_exact_against_the_oracle(n_groups, k, d):
+    """Three rounds of rewiring; after each, the device arrays equal the oracle's
+    stable counting sort of the new index sets."""
+    idx = I.make_idx(n_groups, k, d, 3)
+    plan = H.haste_plan(idx, 32, d)
+    e_idx, e_off, e_ent = plan.export()
+    st, r_off, r_ent = O.plan(idx, d)
+    assert np.array_equal(e_off, r_off) and np.array_equal(e_ent, r_ent)   # the device-built plan
+    for it in range(3):
+        frac = 0.01 if n_groups > 100_000 else 0.05
+        groups, rows, idx = _rewire(idx, d, frac, 0.25 if k > 4 else 0.5, it)
+        plan.update(groups, rows)
+        torch.cuda.synchronize()
+        e_idx, e_off, e_ent = plan.export()
+        st, r_off, r_ent = O.plan(idx, d)
+        assert st == O.OK
+        assert np.array_equal(e_idx, idx), it
+        assert np.array_equal(e_off, r_off) and np.array_equal(e_ent, r_ent), it
+
+
+def test_fused_step_after_a_plan_update_uses_the_new_sets():
+    c = dict(B=130, d=384, n_groups=250, G=32, k=64, dtype="bf16", H=0, p=5)
+    idx, X, W, tpos, _ = _step_inputs(c)
+    plan = H.haste_plan(idx, c["G"], c["d"])
+    groups, rows, idx2 = _rewire(idx, c["d"], 0.3, 0.5, 11)
+    plan.update(groups, rows)
+    scale = 1.0 / c["B"]
+    loss, dW, dX = _run_step(plan, X, W, tpos, scale)
+    assert H.haste_device_status() == H.HASTE_OK
+    r_loss, _, r_dW, r_dX = O.bce_step(X, W, idx2, c["G"], tpos[0], tpos[1], scale)
+    assert abs(float(loss.item()) - r_loss) <= 5e-3 * abs(r_loss)
+    assert_close(to_np64(dW), r_dW, "dW after the update")
+    assert_close(to_np64(dX), r_dX, "dX after the update")
+
+
+def test_plan_update_rejects_bad_edits_and_keeps_the_plan():
+    idx = I.make_idx(50, 16, 64, 2)
+    plan = H.haste_plan(idx, 16, 64)
+    good = np.sort(np.random.default_rng(0).choice(64, 16, replace=False)).astype(np.int32)
+    bad_rows = [good.copy(), good.copy()]
+    bad_rows[0][3] = bad_rows[0][2]                 # a duplicate
+    bad_rows[1][-1] = 64                            # out of range
+    for row, code in zip(bad_rows, (H.HASTE_ERR_INDEX_UNSORTED_OR_DUP, H.HASTE_ERR_INDEX_OUT_OF_RANGE)):
+        with pytest.raises(H.HasteError) as e:
+            plan.update(np.array([4]), row[None, :])
+        assert e.value.status == code
+    for groups in (np.array([5, 5]), np.array([7, 3]), np.array([50])):   # repeated, descending, out of range
+        with pytest.raises(H.HasteError) as e:
+            plan.update(groups, np.tile(good, (len(groups), 1)))
+        assert e.value.status == H.HASTE_ERR_INVALID_ARG
+    e_idx, e_off, e_ent = plan.export()
+    st, r_off, r_ent = O.plan(idx, 64)
+    assert np.array_equal(e_idx, idx) and np.array_equal(e_off, r_off) and np.array_equal(e_ent, r_ent)

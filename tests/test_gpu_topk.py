@@ -65,6 +65,10 @@ CASES = [
     dict(B=256, d=768, n_groups=200, G=64, k=128, K=16, kp=4, nb=50),  # approximate (kp < K)
     dict(B=200, d=512, n_groups=150, G=32, k=128, K=3, kp=1, nb=150),  # one bucket per group
     dict(B=32, d=256, n_groups=64, G=16, k=64, K=64, kp=8, nb=8),      # k = n_buckets * kp
+    # the benchmark's scoring setting: K' = 4 < K = 5, one bucket per SM of a B200,
+    # n_groups not a multiple of the bucket count (uneven buckets of 2 and 3 groups)
+    dict(B=130, d=256, n_groups=333, G=32, k=64, K=5, kp=4, nb=148),
+    dict(B=256, d=768, n_groups=1001, G=32, k=128, K=5, kp=4, nb=148),
 ]
 
 
@@ -84,16 +88,19 @@ def test_topk_matches_oracle(c):
     assert np.array_equal(gi, gi2) and np.array_equal(gv, gv2)
 
 
-def test_topk_full_size_670k_sampled_rows():
+@pytest.mark.parametrize("kp", [8, 4])
+def test_topk_full_size_670k_sampled_rows(kp):
+    """The 670K workload with one bucket per SM (20,944 groups in 148 buckets do not
+    divide evenly); kp = 4 with K = 5 is the benchmark's scoring setting."""
     wl = I.WORKLOADS["670k"]
     idx = I.make_idx(wl.n_groups, wl.k, wl.d, 0)
     X = I.make_normal((wl.B, wl.d), 1.0, 0, 1, "bf16")
     W = I.make_normal((wl.L, wl.k), 1.0 / math.sqrt(wl.k), 0, 2, "bf16")
     plan = H.haste_plan(idx, wl.G, wl.d)
     nb = torch.cuda.get_device_properties(0).multi_processor_count
-    gv, gi = _run(plan, to_torch(X), to_torch(W), 5, 8, nb)
-    rows = np.array([0, 1, 77, wl.B - 1], dtype=np.int32)
-    rv, ri = O.topk(X, W, idx, wl.G, 5, 8, nb, rows=rows)
+    gv, gi = _run(plan, to_torch(X), to_torch(W), 5, kp, nb)
+    rows = np.array([0, 1, 77, 130, wl.B - 1], dtype=np.int32)
+    rv, ri = O.topk(X, W, idx, wl.G, 5, kp, nb, rows=rows)
     true = lambda r, ids: O.logits_at(X, W, idx, wl.G, np.full(len(ids), rows[r], np.int32), ids.astype(np.int64))
     _check(gv[rows], gi[rows], rv, ri, true, wl.L, "670k")
 
