@@ -87,7 +87,6 @@ def algorithmic(wl):
 # source file it was taken on: (config, timed region) -> (bytes, source digest).
 TRAFFIC = {
     ("670k", "tail_step"): (643.1e6, "6c87e65aba6e9fd4"),
-    ("670k", "tail_dx"): (531.9e6, "3a3a2a8a7580d6d9"),
     ("670k", "topk_score"): (186.2e6, "a08fbb472ccd8c70"),
 }
 # timed region -> (source file under csrc/, kernel name in the ncu summaries)

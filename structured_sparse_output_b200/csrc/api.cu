@@ -20,7 +20,6 @@
 #include "tail.cu"
 #include "tail_v2.cu"
 #include "dx_band.cu"
-#include "dx_z.cu"
 #include "tail_given.cu"
 #include "topk.cu"
 #include "plan.cu"
@@ -129,28 +128,29 @@ class ProfScope {
   cudaEvent_t a_ = nullptr;
 };
 
-// Tiling of the dX pass.  ns > 0: the pipelined scatter kernel (k_dx_z) with an
-// ns-stage ring, one CTA per (group chunk, 128-row batch tile, feature part of
-// part_w features); ns = 0: the staged kernel, feature bands sized so the fp32
-// band accumulator fits in shared memory.  Group chunks: as many as keep every
-// CTA resident.
+// Tiling of the dX pass.  ns > 0: the pipelined band-product kernel (k_dx_band)
+// with an ns-stage ring, one CTA per (group chunk, feature band of up to 256,
+// batch half of up to 256 rows); ns = 0: the staged kernel, feature bands sized
+// so the fp32 band accumulator fits in shared memory.  Group chunks: as many as
+// keep every CTA resident.
 struct DxTiling {
-  int band, n_bands, n_chunks, ns, n_parts, part_w;
+  int band, n_bands, n_chunks, ns, n_halves;
 };
 
 // The warp-specialised TMA kernels cover bf16 with G in {16, 32, 64} and k in
 // {64, 128}: the fused step kernel up to two 128-row batch tiles, the dX pass up
 // to four; other shapes run the staged kernels of tail.cu.
 bool use_v2(const haste_plan_s& p, int Bp, int elem) { return elem == 2 && tail2::supported(p.G, p.k, Bp); }
-bool use_dxz(const haste_plan_s& p, int Bp, int elem) { return elem == 2 && tail2::dxz_supported(p.G, p.k, Bp); }
+bool use_dx_band(const haste_plan_s& p, int Bp, int elem) { return elem == 2 && tail2::dx_supported(p.G, p.k, Bp); }
 
 DxTiling dx_tiling(const haste_plan_s& p, int Bp, int elem, int sms, int smem_optin) {
   DxTiling t{};
   const int kHeadroom = 4096;  // static shared memory and launch reserve
   int per_chunk;
-  if (use_dxz(p, Bp, elem) &&
-      tail2::dxz_config(p.G, p.k, p.d, (size_t)smem_optin, kHeadroom, &t.n_parts, &t.part_w, &t.ns)) {
-    per_chunk = (Bp / 128) * t.n_parts;
+  if (use_dx_band(p, Bp, elem) &&
+      tail2::dx_config(p.G, p.k, p.d, Bp, (size_t)smem_optin, kHeadroom, &t.band, &t.n_bands, &t.ns)) {
+    t.n_halves = (Bp + 255) / 256;
+    per_chunk = t.n_bands * t.n_halves;  // a CTA covers up to 256 batch rows of its band
   } else {
     const long avail = (long)smem_optin - (long)tail::smem_dx(elem, p.k, p.G, 0) - kHeadroom;
     int band = (int)std::min<long>(256, avail / 512);
@@ -242,22 +242,25 @@ TailArgs make_args(const haste_plan_s& p, int B) {
   return a;
 }
 
-// dX pass through the pipelined bf16 kernel, from the caller's row-major [B, L]
+// dX pass through a pipelined bf16 kernel, from the caller's row-major [B, L]
 // gradient or from the fused step's group-major buffer [n_groups, Bp, G].
 cudaError_t dx_v2(const haste_plan_s& p, int B, const void* W, const void* dY, bool group_major, float* part,
                   const DxTiling& t, cudaStream_t s) {
-  v2::DxzArgs a{};
+  v2::DxArgs a{};
   a.sh = make_args(p, B).sh;
   a.idx = p.idx_d;
   a.dY = static_cast<const __nv_bfloat16*>(dY);
   a.W = static_cast<const __nv_bfloat16*>(W);
   a.dX_part = part;
+  a.band = t.band;
+  a.n_bands = t.n_bands;
+  a.n_halves = t.n_halves;
   a.n_chunks = t.n_chunks;
-  a.n_parts = t.n_parts;
-  a.part_w = t.part_w;
   a.ns = t.ns;
-  a.dy_group_major = group_major ? 1 : 0;
-  return tail2::launch_dxz(p.G, p.k, a, dY, W, s);
+  // element (b, g*G + j) of dY sits at dY[g*gstride + b*rstride + j]
+  a.dy_gstride = group_major ? (int64_t)a.sh.Bp * p.G : p.G;
+  a.dy_rstride = group_major ? p.G : a.sh.L;
+  return tail2::launch_dx(p.G, p.k, a, dY, W, s);
 }
 
 template <typename T>
@@ -626,7 +629,7 @@ haste_status_t haste_forward(haste_plan_t p, int32_t B, haste_dtype_t dt, const 
   }
   if (e == cudaSuccess) {
     ProfScope ps("tail_forward", s);
-    const int Bp = a.sh.Bp, ns = tail3::stages(p->k, p->G, (size_t)di.smem_optin, 4096);
+    const int Bp = a.sh.Bp, ns = tail3::stages(p->k, p->G, (size_t)di.smem_optin, 4096, true);
     if (dt == HASTE_BF16 && tail3::supported(p->G, p->k, Bp) && ns > 0) {
       v3::GivenArgs g{};
       g.sh = a.sh;
@@ -669,7 +672,7 @@ haste_status_t haste_backward_dw(haste_plan_t p, int32_t B, haste_dtype_t dt, co
   }
   if (e == cudaSuccess) {
     ProfScope ps("tail_dw", s);
-    const int Bp = a.sh.Bp, ns = tail3::stages(p->k, p->G, (size_t)di.smem_optin, 4096);
+    const int Bp = a.sh.Bp, ns = tail3::stages(p->k, p->G, (size_t)di.smem_optin, 4096, false);
     if (dt == HASTE_BF16 && tail3::supported(p->G, p->k, Bp) && ns > 0) {
       v3::GivenArgs g{};
       g.sh = a.sh;

@@ -2,7 +2,7 @@
 // (HASTE, "Hardware-Aware Dynamic Sparse Training for Large Output Spaces",
 // Methodology 1; the dX step of the backward pass).
 //
-// k_dx_band -- per CTA (feature band, group chunk), every batch row: warp 0 loads
+// k_dx_band -- per CTA (feature band, group chunk, batch half of up to 256 rows): warp 0 loads
 //   each group's dY tile and G x k weight block into a shared-memory ring with
 //   TMA, warps 2-9 (two sets of four, alternate groups) densify the weight block
 //   over the band, warp 1 issues one MMA per 128-row batch tile into TMEM
@@ -21,9 +21,11 @@ struct DxArgs {
   const __nv_bfloat16* W;
   float* dX_part;
   int band, n_bands, n_chunks, ns;  // ns: stages of the shared-memory ring
+  int n_halves;                      // batch halves of up to 256 rows (2 when B > 256)
   // element (b, g*G + j) of dY is at dY[g*dy_gstride + b*dy_rstride + j]
   int64_t dy_gstride, dy_rstride;
-  // dY tile of group g (every batch row) in the dY tensor map: x = g*dy_xg, y = g*dy_yg
+  // dY tile of group g (the batch half's rows) in the dY tensor map: x = g*dy_xg,
+  // y = g*dy_yg + 256*half
   int dy_xg, dy_yg;
 };
 
@@ -64,8 +66,8 @@ constexpr int kDxThreads = 320;  // producer warp, MMA warp, two sets of 4 densi
 // one tcgen05 MMA per 128-row batch tile and group (M = 128 batch rows, N = NB,
 // K = G), accumulated in TMEM.  A group's slots hold distinct features, so a
 // (b, f) entry receives exactly that group's term dY_g[b, :] . W_g[:, s].
-// One CTA owns a feature band, every batch row (up to two 128-row TMEM
-// accumulators of NB columns) and a chunk of groups:
+// One CTA owns a feature band, a batch half of up to 256 rows (up to two 128-row
+// TMEM accumulators of NB columns) and a chunk of groups:
 //   producer (warp 0, one thread): the dY tile (Bp x G, K-major, swizzled rows of
 //     2G bytes) and the G x k weight block into a stage of the ring with TMA;
 //   densify (two sets of four warps, warps 2-5 for the even groups of the chunk,
@@ -86,16 +88,18 @@ __global__ void __launch_bounds__(kDxThreads, 1)
   constexpr int RB = kG * 2;  // bytes of a K-major row (G bf16)
   const int NS = a.ns, NB = a.band;
   const TailShape sh = a.sh;
-  const int MT = sh.Bp / 128;
-  const int c = blockIdx.x / a.n_bands;
+  const int BH = min(sh.Bp, 256);  // rows of the dY box (a batch half)
   const int h = blockIdx.x % a.n_bands;
+  const int bh = (blockIdx.x / a.n_bands) % a.n_halves;
+  const int c = blockIdx.x / (a.n_bands * a.n_halves);
+  const int MT = min(2, (sh.Bp - 256 * bh) / 128);  // 128-row tiles of this half
   const int f0 = h * NB;
   const int nf = min(sh.d, f0 + NB) - f0;
   const int64_t g0 = (int64_t)c * sh.n_groups / a.n_chunks;
   const int64_t g1 = (int64_t)(c + 1) * sh.n_groups / a.n_chunks;
   const int n = (int)(g1 - g0);
 
-  const DxLayout Lo = dx_layout(sh.Bp, NB, kK, kG, NS);
+  const DxLayout Lo = dx_layout(BH, NB, kK, kG, NS);
   const uint32_t base = align1024(smem_u32(smem));
   uint8_t* gbase = smem + (base - smem_u32(smem));
   auto DYS = [&](int st) -> uint32_t { return base + Lo.dy + st * Lo.dy_stride; };
@@ -141,12 +145,12 @@ __global__ void __launch_bounds__(kDxThreads, 1)
   if (w == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      const uint32_t bytes = (uint32_t)(sh.Bp + kK) * RB;  // dY tile + weight block
+      const uint32_t bytes = (uint32_t)(BH + kK) * RB;  // dY tile + weight block
       const bool group_major = a.dy_gstride != kG;
       // a ring load from HBM takes longer than the ring's MMA work: the tiles of
       // later groups are requested into L2 ahead of their ring loads
       auto prefetch = [&](int64_t g) {
-        if (group_major) prefetch_l2(a.dY + g * a.dy_gstride, (uint32_t)(sh.Bp * RB));
+        if (group_major) prefetch_l2(a.dY + g * a.dy_gstride + (int64_t)256 * bh * kG, (uint32_t)(BH * RB));
         prefetch_l2(a.W + g * kG * kK, (uint32_t)(kG * kK * 2));
         prefetch_l2(a.idx + g * kK, (uint32_t)(kK * 4));
       };
@@ -158,7 +162,7 @@ __global__ void __launch_bounds__(kDxThreads, 1)
         if (!wait_or_abort(&empty[st], ph ^ 1, abort_flag)) break;
         ++issued;
         mbar_arrive_expect_tx(&full[st], bytes);
-        tma_load_2d(DYS(st), &tm_dy, (int)(g * a.dy_xg), (int)(g * a.dy_yg), &full[st]);
+        tma_load_2d(DYS(st), &tm_dy, (int)(g * a.dy_xg), (int)(g * a.dy_yg + 256 * bh), &full[st]);
 #pragma unroll
         for (int blk = 0; blk < kK / 64; ++blk)
           tma_load_2d(WS(st) + (uint32_t)(blk * kG * 128), &tm_w, 64 * blk, (int)(g * kG), &full[st]);
@@ -277,7 +281,7 @@ __global__ void __launch_bounds__(kDxThreads, 1)
     if (fin) {
       // two batch tiles: one per set; one tile: the sets take alternate 16-column chunks
       for (int t = MT == 2 ? set : 0; t < (MT == 2 ? set + 1 : 1); ++t) {
-        const int b = t * 128 + q * 32 + lane;
+        const int b = 256 * bh + t * 128 + q * 32 + lane;
         for (int c0 = MT == 2 ? 0 : 16 * set; c0 < NB; c0 += MT == 2 ? 16 : 32) {
           float v[16];
           tmem_ld16(tmem + lane_off + (uint32_t)(t * 256 + c0), v);
@@ -309,7 +313,12 @@ size_t dx_smem(int Bp, int band, int k, int G, int ns) { return v2::dx_layout(Bp
 // (the widest MMA N), as few as cover d, split evenly in multiples of 16; the
 // deepest ring (up to six stages) that fits in the shared memory left after
 // `reserve` bytes.  Returns false when two stages do not fit.
+bool dx_supported(int G, int k, int Bp) {
+  return (G == 16 || G == 32 || G == 64) && (k == 64 || k == 128) && Bp <= 512;
+}
+
 bool dx_config(int G, int k, int d, int Bp, size_t smem_optin, size_t reserve, int* band, int* n_bands, int* ns) {
+  Bp = Bp < 256 ? Bp : 256;  // a CTA covers a batch half of up to 256 rows
   const int nb = (d + 255) / 256;
   const int bw = (((d + nb - 1) / nb) + 15) & ~15;
   int best = 0;
@@ -328,24 +337,25 @@ bool dx_config(int G, int k, int d, int Bp, size_t smem_optin, size_t reserve, i
 // tensor and read as zeros).
 template <int kG, int kK>
 cudaError_t launch_dx_t(v2::DxArgs a, const void* dY, const void* W, cudaStream_t st) {
-  const size_t smem = dx_smem(a.sh.Bp, a.band, kK, kG, a.ns);
+  const int BH = a.sh.Bp < 256 ? a.sh.Bp : 256;
+  const size_t smem = dx_smem(BH, a.band, kK, kG, a.ns);
   auto kern = v2::k_dx_band<kG, kK>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   CUtensorMap tm_dy, tm_w;
   const bool group_major = a.dy_gstride != kG;  // row-major [B, L] has dy_gstride = G
   if (group_major) {
-    e = tmap_2d(&tm_dy, dY, kG, (uint64_t)a.sh.n_groups * a.sh.Bp, (uint64_t)kG * 2, kG, (uint32_t)a.sh.Bp);
+    e = tmap_2d(&tm_dy, dY, kG, (uint64_t)a.sh.n_groups * a.sh.Bp, (uint64_t)kG * 2, kG, (uint32_t)BH);
     a.dy_xg = 0;
     a.dy_yg = a.sh.Bp;
   } else {
-    e = tmap_2d(&tm_dy, dY, (uint64_t)a.sh.L, (uint64_t)a.sh.B, (uint64_t)a.dy_rstride * 2, kG, (uint32_t)a.sh.Bp);
+    e = tmap_2d(&tm_dy, dY, (uint64_t)a.sh.L, (uint64_t)a.sh.B, (uint64_t)a.dy_rstride * 2, kG, (uint32_t)BH);
     a.dy_xg = kG;
     a.dy_yg = 0;
   }
   if (e == cudaSuccess) e = tmap_2d(&tm_w, W, kK, (uint64_t)a.sh.L, (uint64_t)kK * 2, 64, kG);
   if (e != cudaSuccess) return e;
-  const int grid = a.n_bands * a.n_chunks;
+  const int grid = a.n_bands * a.n_halves * a.n_chunks;
   kern<<<grid, v2::kDxThreads, smem, st>>>(a, tm_dy, tm_w);
   return cudaGetLastError();
 }

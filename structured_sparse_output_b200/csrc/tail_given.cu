@@ -10,8 +10,10 @@
 //              warps 0 and 2 fill the even items, 1 and 3 the odd ones;
 //   warp 4     MMA: logits tile (M = 128 batch rows, N = G, K = k) into a 2-deep
 //              TMEM ring;
-//   warps 5-8  epilogue: thread = batch row; the G logits of its row, as bf16, in
-//              16-byte stores.
+//   warps 5-8  epilogue: thread = batch row; the G logits of its row, as bf16, into
+//              a shared-memory staging tile; each warp writes its 32 rows to
+//              global memory with one TMA store (logits rows are L apart, so
+//              per-thread stores would touch 32 rows per instruction).
 // k_dw3 -- one CTA per group chunk, every batch row; items are (group, batch tile):
 //   warps 0-3  producers: the gathered tile of the item and its dY tile (128 rows
 //              x G, rows past B read as zeros), cp.async into a ring;
@@ -42,11 +44,12 @@ constexpr int kGivenMaxStages = 6;
 
 // Shared memory: ns stages of (gathered tile [2 b-blocks][k rows + pad][128 B],
 // second operand: weight block [k/64][G][128 B] (forward) or dY tile
-// [128][2G B] (dW)), then the barriers.
+// [128][2G B] (dW)), for the forward two staging tiles of the output
+// [128][2G B], then the barriers.
 struct GivenLayout {
-  uint32_t xg_stride, op_stride, xg, op, bars, total;
+  uint32_t xg_stride, op_stride, out_stride, xg, op, out, bars, total;
 };
-__host__ __device__ inline GivenLayout given_layout(int k, int G, int ns) {
+__host__ __device__ inline GivenLayout given_layout(int k, int G, int ns, bool fwd) {
   GivenLayout L;
   // 2 b-blocks of k rows; rows k..127 of the last block are padding that an
   // M = 128 product reads when k = 64 (those TMEM lanes are not read out)
@@ -58,6 +61,9 @@ __host__ __device__ inline GivenLayout given_layout(int k, int G, int ns) {
   off += ns * L.xg_stride;
   L.op = off;
   off += ns * L.op_stride;
+  L.out_stride = fwd ? (uint32_t)((128 * G * 2 + 1023) & ~1023) : 0u;
+  L.out = off;
+  off += 2 * L.out_stride;
   L.bars = off;
   off += 256;
   L.total = off + 1024;
@@ -92,7 +98,7 @@ __device__ __forceinline__ void load_rows(int (&rows_idx)[kK / 8], const int32_t
 
 // ============================================================ k_fwd3
 template <int kG, int kK>
-__global__ void __launch_bounds__(kGivenThreads, 1) k_fwd3(GivenArgs a) {
+__global__ void __launch_bounds__(kGivenThreads, 1) k_fwd3(GivenArgs a, const __grid_constant__ CUtensorMap tm_out) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const TailShape sh = a.sh;
   const int NS = a.ns;
@@ -100,7 +106,7 @@ __global__ void __launch_bounds__(kGivenThreads, 1) k_fwd3(GivenArgs a) {
   const int c = blockIdx.x / n_bt, t = blockIdx.x % n_bt;
   const int64_t gb = (int64_t)c * sh.n_groups / a.n_chunks;
   const int n_items = (int)((int64_t)(c + 1) * sh.n_groups / a.n_chunks - gb);
-  const GivenLayout Lo = given_layout(kK, kG, NS);
+  const GivenLayout Lo = given_layout(kK, kG, NS, true);
   const uint32_t base = align1024(smem_u32(smem));
   uint8_t* gbase = smem + (base - smem_u32(smem));
   uint64_t* bars = reinterpret_cast<uint64_t*>(gbase + Lo.bars);
@@ -187,33 +193,43 @@ __global__ void __launch_bounds__(kGivenThreads, 1) k_fwd3(GivenArgs a) {
     (void)__all_sync(0xffffffffu, mbar_wait(done, 0));
   } else {
     // ------------------------------------------------------------- epilogue
+    constexpr int RB = kG * 2;  // bytes of an output row
     const int q = w & 3;
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-    const int b = t * 128 + q * 32 + lane;
-    const bool live = b < sh.B;
+    const int r = q * 32 + lane;                      // row of the batch tile
+    const bool warp_rows = t * 128 + q * 32 < sh.B;  // some of this warp's rows are inside the batch
     for (int i = 0; i < n_items; ++i) {
       const int fb = i & 1;
+      // this warp's store from the same staging tile two items ago has read it
+      if (lane == 0) bulk_wait_read<1>();
+      __syncwarp();
       if (!__all_sync(0xffffffffu, wait_or_abort(&f_full[fb], (i >> 1) & 1, abort_flag))) break;
       tc_fence_after();
-      __nv_bfloat16* dst = a.out + (int64_t)b * sh.L + (gb + i) * kG;
+      float vall[kG];
 #pragma unroll
-      for (int c0 = 0; c0 < kG; c0 += 16) {
-        float v[16];
-        tmem_ld16(tmem + lane_off + (uint32_t)(fb * kG + c0), v);
-        tmem_wait_ld();
-        if (live) {
-          const uint4 lo = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
-                                      pack_bf16x2(v[6], v[7]));
-          const uint4 hi = make_uint4(pack_bf16x2(v[8], v[9]), pack_bf16x2(v[10], v[11]),
-                                      pack_bf16x2(v[12], v[13]), pack_bf16x2(v[14], v[15]));
-          *reinterpret_cast<uint4*>(dst + c0) = lo;
-          *reinterpret_cast<uint4*>(dst + c0 + 8) = hi;
-        }
-      }
+      for (int c0 = 0; c0 < kG; c0 += 16)
+        tmem_ld16(tmem + lane_off + (uint32_t)(fb * kG + c0), *reinterpret_cast<float(*)[16]>(&vall[c0]));
+      tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&f_empty[fb]);
+      if (lane == 0) mbar_arrive(&f_empty[fb]);  // TMEM read: the next product may overwrite it
+      uint8_t* out = gbase + Lo.out + fb * Lo.out_stride;
+#pragma unroll
+      for (int c0 = 0; c0 < kG; c0 += 8) {
+        const float* v = &vall[c0];
+        const uint4 pk = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                                    pack_bf16x2(v[6], v[7]));
+        *reinterpret_cast<uint4*>(out + swz_rows((uint32_t)(r * RB + c0 * 2), RB)) = pk;
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0 && warp_rows) {
+        tma_store_2d(&tm_out, base + Lo.out + fb * Lo.out_stride + (uint32_t)(q * 32 * RB), (int)((gb + i) * kG),
+                     t * 128 + q * 32);
+        bulk_commit();
+      }
     }
+    if (lane == 0) bulk_wait_all();  // the stores are complete before the CTA exits
   }
   tc_fence_before();
   __syncthreads();
@@ -234,7 +250,7 @@ __global__ void __launch_bounds__(kGivenThreads, 1) k_dw3(GivenArgs a) {
   const int64_t gb = (int64_t)blockIdx.x * sh.n_groups / a.n_chunks;
   const int n_groups = (int)((int64_t)(blockIdx.x + 1) * sh.n_groups / a.n_chunks - gb);
   const int n_items = n_groups * n_bt;  // item i: group i / n_bt, batch tile i % n_bt
-  const GivenLayout Lo = given_layout(kK, kG, NS);
+  const GivenLayout Lo = given_layout(kK, kG, NS, false);
   const uint32_t base = align1024(smem_u32(smem));
   uint8_t* gbase = smem + (base - smem_u32(smem));
   uint64_t* bars = reinterpret_cast<uint64_t*>(gbase + Lo.bars);
@@ -331,11 +347,14 @@ __global__ void __launch_bounds__(kGivenThreads, 1) k_dw3(GivenArgs a) {
       if (!__all_sync(0xffffffffu, wait_or_abort(&d_full[db], (gi >> 1) & 1, abort_flag))) break;
       tc_fence_after();
       const int64_t g = gb + gi;
+      float vall[kG];
+#pragma unroll
+      for (int c0 = 0; c0 < kG; c0 += 16)
+        tmem_ld16(tmem + lane_off + (uint32_t)(db * kG + c0), *reinterpret_cast<float(*)[16]>(&vall[c0]));
+      tmem_wait_ld();
 #pragma unroll
       for (int c0 = 0; c0 < kG; c0 += 16) {
-        float v[16];
-        tmem_ld16(tmem + lane_off + (uint32_t)(db * kG + c0), v);
-        tmem_wait_ld();
+        const float* v = &vall[c0];
         if (r < kK) {
           __nv_bfloat16* dst = a.out + (g * kG + c0) * kK + r;  // lanes: consecutive slots
 #pragma unroll
@@ -364,29 +383,33 @@ bool supported(int G, int k, int Bp) {
   return (G == 16 || G == 32 || G == 64) && (k == 64 || k == 128) && Bp <= 512;
 }
 
-size_t smem_for(int k, int G, int ns) { return v3::given_layout(k, G, ns).total; }
+size_t smem_for(int k, int G, int ns, bool fwd) { return v3::given_layout(k, G, ns, fwd).total; }
 
 // Deepest ring (2 to 6 stages) that fits; 0 when two stages do not.
-int stages(int k, int G, size_t smem_optin, size_t reserve) {
+int stages(int k, int G, size_t smem_optin, size_t reserve, bool fwd) {
   int best = 0;
   for (int st = 2; st <= v3::kGivenMaxStages; ++st)
-    if (smem_for(k, G, st) + reserve <= smem_optin) best = st;
+    if (smem_for(k, G, st, fwd) + reserve <= smem_optin) best = st;
   return best;
 }
 
 template <int kG, int kK>
 cudaError_t launch_fwd_t(const v3::GivenArgs& a, cudaStream_t st) {
-  const size_t smem = smem_for(kK, kG, a.ns);
+  const size_t smem = smem_for(kK, kG, a.ns, true);
   auto kern = v3::k_fwd3<kG, kK>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  kern<<<a.n_chunks * (a.sh.Bp / 128), v3::kGivenThreads, smem, st>>>(a);
+  // the logits [B, L] as the stores' tensor: boxes of G labels x 32 rows
+  CUtensorMap tm_out;
+  e = tail2::tmap_2d(&tm_out, a.out, (uint64_t)a.sh.L, (uint64_t)a.sh.B, (uint64_t)a.sh.L * 2, kG, 32);
+  if (e != cudaSuccess) return e;
+  kern<<<a.n_chunks * (a.sh.Bp / 128), v3::kGivenThreads, smem, st>>>(a, tm_out);
   return cudaGetLastError();
 }
 
 template <int kG, int kK>
 cudaError_t launch_dw_t(const v3::GivenArgs& a, cudaStream_t st) {
-  const size_t smem = smem_for(kK, kG, a.ns);
+  const size_t smem = smem_for(kK, kG, a.ns, false);
   auto kern = v3::k_dw3<kG, kK>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;

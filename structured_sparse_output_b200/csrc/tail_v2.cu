@@ -9,7 +9,7 @@
 //   warp 4     MMA issuer (one thread): issues each group's forward and dW
 //              product as soon as its inputs are ready, so the tensor core works
 //              while the epilogue runs;
-//   warps 5-20 epilogue: logits leave TMEM only as the BCE gradient (bf16, to
+//   warps 5-12 epilogue: logits leave TMEM only as the BCE gradient (bf16, to
 //              shared memory for the dW product and to the group-major gradient
 //              buffer of the dX pass); the BCE of group i+1 comes before the dW
 //              readout of group i, so the dW product runs behind it.  The readout
@@ -82,7 +82,7 @@ __device__ __forceinline__ void publish_all(uint64_t* full_bar) {
 // ============================================================ k_step2
 constexpr int kStepProd = 4;       // producer warps: two per ring stage
 constexpr int kStepMma = kStepProd;  // warp id of the MMA issuer
-constexpr int kStepEpi = 16;       // epilogue warps: 4 lane quarters x 2 column halves x 2 batch tiles
+constexpr int kStepEpi = 8;        // epilogue warps: 4 lane quarters x 2 column halves
 constexpr int kStepThreads = 32 * (kStepProd + 1 + kStepEpi);  // producers, MMA warp, epilogue warps
 constexpr int kMaxPosReg = 8;      // positives per batch row kept in registers
 
@@ -166,6 +166,7 @@ __global__ void __launch_bounds__(kStepThreads, 1)
       if (part == 0 && lane == 0 && i + 2 < n_items) {
         prefetch_l2(W + (g + 2) * kG * kK, (uint32_t)(kG * kK * 2));
         prefetch_l2(a.idx + (g + 2) * kK, (uint32_t)(kK * 4));
+        if constexpr (kUpd == 2) prefetch_l2(a.M + (g + 2) * kG * kK, (uint32_t)(kG * kK * 2));  // read by the update
       }
       // the index loads are in flight while this half waits for its stage
       int idx_cur[kRows];
@@ -279,54 +280,67 @@ __global__ void __launch_bounds__(kStepThreads, 1)
     (void)__all_sync(0xffffffffu, mbar_wait(done, 0));
   } else {
     // ------------------------------------------------------------- epilogue
-    // warp (q, hh, tt): TMEM lane quarter q.  BCE: batch tile tt, label columns
-    // [hh*CH, hh*CH + CH) (warps of a tile beyond the batch only take part in the
-    // barriers).  dW readout: slots 32q.., label columns [hh*CH + tt*RC, +RC).
-    constexpr int RC = CH / 2;
-    const int ew = w - kStepMma - 1, q = w & 3, hh = (ew >> 2) & 1, tt = ew >> 3;
+    // warp (q, hh): TMEM lane quarter q, label columns [hh*CH, hh*CH + CH)
+    const int ew = w - kStepMma - 1, q = w & 3, hh = ew >> 2;
     const int r = q * 32 + lane;  // row inside a 128-row tile (and dW slot)
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     const float scale = a.grad_scale;
-    const bool has_tile = tt < n_bt;
-    const int b = tt * 128 + r;
-    const bool live = has_tile && b < sh.B;
     float loss_acc = 0.f;
-    // this thread's positives (tail-local ids)
-    int pos[kMaxPosReg];
-    int npos = 0, pbeg = 0;
-    if (live) {
-      pbeg = a.pos_ptr[b];
-      npos = a.pos_ptr[b + 1] - pbeg;
-    }
+    // this thread's positives (tail-local ids), one batch row per 128-row tile
+    int pos[2][kMaxPosReg];
+    int npos[2] = {0, 0}, pbeg[2] = {0, 0};
 #pragma unroll
-    for (int e = 0; e < kMaxPosReg; ++e) pos[e] = e < npos ? a.pos_ids[pbeg + e] : -1;
+    for (int t = 0; t < 2; ++t) {
+      const int b = t * 128 + r;
+      if (t < n_bt && b < sh.B) {
+        pbeg[t] = a.pos_ptr[b];
+        npos[t] = a.pos_ptr[b + 1] - pbeg[t];
+      }
+#pragma unroll
+      for (int e = 0; e < kMaxPosReg; ++e) pos[t][e] = e < npos[t] ? a.pos_ids[pbeg[t] + e] : -1;
+    }
     auto bce = [&](int i) -> bool {
       const int64_t g = gb + i;
       const int s = i & 1;
       if (!wait_or_abort(&fwd_full[s], (i >> 1) & 1, abort_flag)) return false;
       tc_fence_after();
-      if (has_tile) {
-        const int64_t l0 = g * kG + hh * CH;  // first label of this warp's columns
-        uint8_t* dyrow = gbase + DY(s);
-        __nv_bfloat16* dyg = a.dY_out + g * (int64_t)Bp * kG;
+      const int64_t l0 = g * kG + hh * CH;  // first label of this warp's columns
+      uint8_t* dyrow = gbase + DY(s);
+      __nv_bfloat16* dyg = a.dY_out + g * (int64_t)Bp * kG;
+      // every logit of this thread's columns in both batch tiles is requested from
+      // TMEM before the first is used: one load latency per group, not one per chunk
+      constexpr int NC = CH < 16 ? CH : 16;
+      float zall[2][CH];
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        if (t < n_bt) {
+#pragma unroll
+          for (int c = 0; c < CH; c += 16) {
+            if constexpr (NC == 8) tmem_ld8(F(s) + lane_off + (uint32_t)(t * kG + hh * CH + c), &zall[t][c]);
+            else tmem_ld16(F(s) + lane_off + (uint32_t)(t * kG + hh * CH + c), *reinterpret_cast<float(*)[16]>(&zall[t][c]));
+          }
+        }
+      }
+      tmem_wait_ld();
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        if (t >= n_bt) break;
+        const int b = t * 128 + r;
+        const bool live = b < sh.B;
         const float sl = live ? scale : 0.f, hs = 0.5f * sl;  // rows beyond B get dY = 0
         uint32_t ym = 0;
 #pragma unroll
         for (int e = 0; e < kMaxPosReg; ++e) {
-          const int64_t l = (int64_t)pos[e] - l0;
-          if (pos[e] >= 0 && l >= 0 && l < CH) ym |= 1u << l;
+          const int64_t l = (int64_t)pos[t][e] - l0;
+          if (pos[t][e] >= 0 && l >= 0 && l < CH) ym |= 1u << l;
         }
-        for (int e = kMaxPosReg; e < npos; ++e) {  // rows with many positives
-          const int64_t l = (int64_t)a.pos_ids[pbeg + e] - l0;
+        for (int e = kMaxPosReg; e < npos[t]; ++e) {  // rows with many positives
+          const int64_t l = (int64_t)a.pos_ids[pbeg[t] + e] - l0;
           if (l >= 0 && l < CH) ym |= 1u << l;
         }
 #pragma unroll
         for (int c = 0; c < CH; c += 16) {
-          constexpr int NC = CH < 16 ? CH : 16;
-          float z[16];
-          if constexpr (NC == 8) tmem_ld8(F(s) + lane_off + (uint32_t)(tt * kG + hh * CH + c), z);
-          else tmem_ld16(F(s) + lane_off + (uint32_t)(tt * kG + hh * CH + c), z);
-          tmem_wait_ld();
+          const float* z = &zall[t][c];
           // y = 0 everywhere first (positives are rare), then the few positive
           // columns are corrected: dY -= scale, loss -= z.
           float dyv[16], relu = 0.f, prod = 1.f;
@@ -370,32 +384,58 @@ __global__ void __launch_bounds__(kStepThreads, 1)
     auto readout = [&](int i) -> bool {
       const int64_t g = gb + i;
       const int s = i & 1;
+      // the update's first W and momentum values do not depend on dW: their loads
+      // are in flight while the dW product finishes
+      constexpr int NC0 = CH < 16 ? CH : 16;
+      float wv0[NC0], mv0[NC0];
+      if constexpr (kUpd > 0) {
+        if (r < kK) {
+          const int64_t o = (g * kG + hh * CH) * kK + r;
+#pragma unroll
+          for (int e = 0; e < NC0; ++e) {
+            wv0[e] = __bfloat162float(W[o + (int64_t)e * kK]);
+            mv0[e] = kUpd == 2 ? __bfloat162float(a.M[o + (int64_t)e * kK]) : 0.f;
+          }
+        }
+      }
       if (!wait_or_abort(&dw_full[s], (i >> 1) & 1, abort_flag)) return false;
       tc_fence_after();
-      // dW readout: row = slot r, columns = this warp's RC labels
-      const int c0 = hh * CH + tt * RC;
-      float v[16];
-      if constexpr (RC == 16) tmem_ld16(D(s) + lane_off + (uint32_t)c0, v);
-      else if constexpr (RC == 8) tmem_ld8(D(s) + lane_off + (uint32_t)c0, v);
-      else tmem_ld4(D(s) + lane_off + (uint32_t)c0, v);
+      // dW readout: row = slot r, columns = this warp's labels (all requested before the wait)
+      constexpr int NCR = CH < 16 ? CH : 16;
+      float vall[CH];
+#pragma unroll
+      for (int c = 0; c < CH; c += 16) {
+        if constexpr (NCR == 8) tmem_ld8(D(s) + lane_off + (uint32_t)(hh * CH + c), &vall[c]);
+        else tmem_ld16(D(s) + lane_off + (uint32_t)(hh * CH + c), *reinterpret_cast<float(*)[16]>(&vall[c]));
+      }
       tmem_wait_ld();
-      if (r < kK) {
-        const int64_t off0 = (g * kG + c0) * kK + r;  // (label, slot r); lanes: consecutive slots
-        if constexpr (kUpd == 0) {
 #pragma unroll
-          for (int e = 0; e < RC; ++e) a.dW[off0 + (int64_t)e * kK] = __float2bfloat16_rn(v[e]);
-        } else {
-          float wv[RC], mv[RC];
+      for (int c = 0; c < CH; c += 16) {
+        constexpr int NC = NCR;
+        const float* v = &vall[c];
+        if (r < kK) {
+          const int64_t off0 = (g * kG + hh * CH + c) * kK + r;  // (label, slot r); lanes: consecutive slots
+          if constexpr (kUpd == 0) {
 #pragma unroll
-          for (int e = 0; e < RC; ++e) {
-            wv[e] = __bfloat162float(W[off0 + (int64_t)e * kK]);
-            mv[e] = kUpd == 2 ? __bfloat162float(a.M[off0 + (int64_t)e * kK]) : 0.f;
-          }
+            for (int e = 0; e < NC; ++e) a.dW[off0 + (int64_t)e * kK] = __float2bfloat16_rn(v[e]);
+          } else {
+            float wv[16], mv[16];
 #pragma unroll
-          for (int e = 0; e < RC; ++e) {
-            const float m = kUpd == 2 ? fmaf(a.momentum, mv[e], v[e]) : v[e];
-            if constexpr (kUpd == 2) a.M[off0 + (int64_t)e * kK] = __float2bfloat16_rn(m);
-            a.W_out[off0 + (int64_t)e * kK] = __float2bfloat16_rn(fmaf(-a.lr, m, wv[e]));
+            for (int e = 0; e < NC; ++e) {
+              if (c == 0) {
+                wv[e] = wv0[e];
+                mv[e] = mv0[e];
+              } else {
+                wv[e] = __bfloat162float(W[off0 + (int64_t)e * kK]);
+                mv[e] = kUpd == 2 ? __bfloat162float(a.M[off0 + (int64_t)e * kK]) : 0.f;
+              }
+            }
+#pragma unroll
+            for (int e = 0; e < NC; ++e) {
+              const float m = kUpd == 2 ? fmaf(a.momentum, mv[e], v[e]) : v[e];
+              if constexpr (kUpd == 2) a.M[off0 + (int64_t)e * kK] = __float2bfloat16_rn(m);
+              a.W_out[off0 + (int64_t)e * kK] = __float2bfloat16_rn(fmaf(-a.lr, m, wv[e]));
+            }
           }
         }
       }

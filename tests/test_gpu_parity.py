@@ -287,9 +287,9 @@ def test_short_wait_limit_reaches_the_abort_paths_and_the_context_survives():
 
 
 SGD_CASES = [
-    dict(B=256, d=768, n_groups=300, G=64, k=128, dtype="bf16", H=0, p=8, lr=4.0, mu=0.9),
-    dict(B=130, d=384, n_groups=250, G=32, k=64, dtype="bf16", H=0, p=5, lr=2.0, mu=0.0),
-    dict(B=100, d=256, n_groups=120, G=16, k=64, dtype="bf16", H=0, p=5, lr=3.0, mu=0.5),
+    dict(B=256, d=768, n_groups=300, G=64, k=128, dtype="bf16", H=0, p=8, lr=8.0, mu=0.9),
+    dict(B=130, d=384, n_groups=250, G=32, k=64, dtype="bf16", H=0, p=5, lr=16.0, mu=0.0),
+    dict(B=100, d=256, n_groups=120, G=16, k=64, dtype="bf16", H=0, p=5, lr=12.0, mu=0.5),
 ]
 
 
@@ -298,8 +298,10 @@ def test_fused_step_with_sgd_update_two_steps(case):
     """haste_bce_step_sgd over two steps, alternating two weight buffers as a
     training loop does: the loss and dX of each step use that step's input
     weights, the momentum buffer and the new weights follow the oracle's SGD
-    update.  lr is large so that the update, not the bf16 rounding of W', decides
-    the comparison of W' - W."""
+    update.  lr is large, so that the update dominates W' and the bf16 rounding
+    of W' (about 2^-9 of W' in relative terms) stays well inside the tolerance on
+    W' - W; with an update the size of W, that rounding alone is about half the
+    rel-L2 tolerance."""
     idx, X, W0, tpos, _ = _step_inputs(case)
     B, d, G, k = case["B"], case["d"], case["G"], case["k"]
     lr, mu = case["lr"], case["mu"]
@@ -373,7 +375,7 @@ def _rewire(idx, d, frac_groups, frac_slots, seed):
     return groups, rows, out
 
 
-@pytest.mark.parametrize("n_groups,k,d", [(20_944, 128, 768), (1000, 64, 97), (7, 5, 5), (134_376, 128, 768)])
+@pytest.mark.parametrize("n_groups,k,d", [(20_944, 128, 768), (1000, 64, 97), (7, 3, 5), (134_376, 128, 768)])
 def test_plan_update_is_bit_exact_against_the_oracle(n_groups, k, d):
     """Three rounds of rewiring; after each, the device arrays equal the oracle's
     stable counting sort of the new index sets."""
@@ -384,7 +386,7 @@ def test_plan_update_is_bit_exact_against_the_oracle(n_groups, k, d):
     assert np.array_equal(e_off, r_off) and np.array_equal(e_ent, r_ent)   # the device-built plan
     for it in range(3):
         frac = 0.01 if n_groups > 100_000 else 0.05
-        groups, rows, idx = _rewire(idx, d, frac, 0.25 if k > 4 else 0.5, it)
+        groups, rows, idx = _rewire(idx, d, frac, 0.25 if k > 4 else 0.34, it)
         plan.update(groups, rows)
         torch.cuda.synchronize()
         e_idx, e_off, e_ent = plan.export()

@@ -110,13 +110,16 @@ def test_topk_argument_errors():
     plan = H.haste_plan(idx, 32, 256)
     X = torch.zeros((8, 256), dtype=torch.bfloat16, device="cuda")
     W = torch.zeros((40 * 32, 64), dtype=torch.bfloat16, device="cuda")
-    ov = torch.empty((8, 4), device="cuda")
-    oi = torch.empty((8, 4), dtype=torch.int32, device="cuda")
     ws = torch.empty(H.haste_topk_workspace_size(plan, 8, H.HASTE_BF16, 4, 2), dtype=torch.uint8, device="cuda")
     for K, kp, nb, code in ((4, 3, 4, H.HASTE_ERR_UNSUPPORTED_SHAPE),   # kp not a power of two <= 8
                             (9, 2, 4, H.HASTE_ERR_INVALID_ARG),         # k > n_buckets * kp
                             (4, 2, 0, H.HASTE_ERR_INVALID_ARG),         # no bucket
                             (4, 2, 41, H.HASTE_ERR_INVALID_ARG)):       # more buckets than groups
+        ov = torch.empty((8, K), device="cuda")
+        oi = torch.empty((8, K), dtype=torch.int32, device="cuda")
         with pytest.raises(H.HasteError) as e:
             H.haste_topk(plan, X, W, K, kp, nb, ov, oi, ws)
         assert e.value.status == code
+    with pytest.raises(ValueError):                                      # outputs not [B, k]: refused by the binding
+        H.haste_topk(plan, X, W, 9, 2, 4, torch.empty((8, 4), device="cuda"),
+                     torch.empty((8, 4), dtype=torch.int32, device="cuda"), ws)
