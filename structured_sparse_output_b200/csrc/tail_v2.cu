@@ -9,10 +9,11 @@
 //   warp 4     MMA issuer (one thread): issues each group's forward and dW
 //              product as soon as its inputs are ready, so the tensor core works
 //              while the epilogue runs;
-//   warps 5-12 epilogue: logits leave TMEM only as the BCE gradient (bf16, to
-//              shared memory for the dW product and to the group-major gradient
-//              buffer of the dX pass); the BCE of group i+1 comes before the dW
-//              readout of group i, so the dW product runs behind it.  The readout
+//   warps 5-12 epilogue: logits leave TMEM only as the BCE gradient (bf16, into
+//              shared memory: the dW operand, and the tile that the MMA thread
+//              writes to the group-major gradient buffer of the dX pass with one
+//              TMA store); the BCE of group i+1 comes before the dW readout of
+//              group i, so the dW product runs behind it.  The readout
 //              writes dW, or (kUpd > 0) applies an SGD update to the group's
 //              weights while dW is on chip: M' = momentum * M + dW (kUpd = 2) or
 //              M' = dW (kUpd = 1), W' = W - lr * M', with W' written to a
@@ -88,7 +89,8 @@ constexpr int kMaxPosReg = 8;      // positives per batch row kept in registers
 
 template <int kG, int kK, int kUpd>
 __global__ void __launch_bounds__(kStepThreads, 1)
-    k_step2(StepArgs a, const __nv_bfloat16* __restrict__ Xt, const __nv_bfloat16* __restrict__ W) {
+    k_step2(StepArgs a, const __nv_bfloat16* __restrict__ Xt, const __nv_bfloat16* __restrict__ W,
+            const __grid_constant__ CUtensorMap tm_dy) {
   extern __shared__ __align__(1024) uint8_t smem[];
   constexpr int RB = kG * 2;   // bytes of one dY row in shared memory
   constexpr int CH = kG / 2;   // label columns per epilogue half
@@ -227,6 +229,10 @@ __global__ void __launch_bounds__(kStepThreads, 1)
                     make_sdesc(WG(s) + (uint32_t)((kk / 4) * kG * 128 + (kk % 4) * 32), 16, 1024, kLayoutSw128);
                 mma_ss<false>(F(s) + (uint32_t)(t * kG), ad, bd, idesc_f, kk > 0 ? 1u : 0u);
               }
+            // the BCE of this group rewrites the dY tile of group nf - 2, whose
+            // store may be the latest one issued: every store must have read its
+            // tile before the BCE is released (the forward's MMAs run meanwhile)
+            bulk_wait_read<0>();
             mma_commit(&fwd_full[s]);
           }
           __syncwarp();
@@ -253,6 +259,9 @@ __global__ void __launch_bounds__(kStepThreads, 1)
             }
             mma_commit(&dw_full[s]);
             mma_commit(&empty[s]);
+            // the group's gradient tile to the dX pass's group-major buffer
+            tma_store_2d(&tm_dy, base + DY(s), 0, (int)((gb + nd) * Bp));
+            bulk_commit();
           }
           __syncwarp();
           ++nd;
@@ -274,8 +283,12 @@ __global__ void __launch_bounds__(kStepThreads, 1)
       }
     }
     // Also after an abort: the CTA frees TMEM and exits only once every MMA it
-    // issued has finished writing TMEM and reading shared memory.
-    if (lane == 0) mma_commit(done);
+    // issued has finished writing TMEM and reading shared memory, and its stores
+    // are complete.
+    if (lane == 0) {
+      mma_commit(done);
+      bulk_wait_all();
+    }
     __syncwarp();
     (void)__all_sync(0xffffffffu, mbar_wait(done, 0));
   } else {
@@ -306,7 +319,6 @@ __global__ void __launch_bounds__(kStepThreads, 1)
       tc_fence_after();
       const int64_t l0 = g * kG + hh * CH;  // first label of this warp's columns
       uint8_t* dyrow = gbase + DY(s);
-      __nv_bfloat16* dyg = a.dY_out + g * (int64_t)Bp * kG;
       // every logit of this thread's columns in both batch tiles is requested from
       // TMEM before the first is used: one load latency per group, not one per chunk
       constexpr int NC = CH < 16 ? CH : 16;
@@ -370,8 +382,7 @@ __global__ void __launch_bounds__(kStepThreads, 1)
                                        pack_bf16x2(dyv[8 * hq + 4], dyv[8 * hq + 5]),
                                        pack_bf16x2(dyv[8 * hq + 6], dyv[8 * hq + 7]));
             const int col = hh * CH + c + 8 * hq;
-            *reinterpret_cast<uint4*>(dyrow + swz_rows((uint32_t)(b * RB + col * 2), RB)) = v;
-            *reinterpret_cast<uint4*>(dyg + (int64_t)b * kG + col) = v;  // rows past B: zeros
+            *reinterpret_cast<uint4*>(dyrow + swz_rows((uint32_t)(b * RB + col * 2), RB)) = v;  // rows past B: zeros
           }
         }
       }
@@ -479,14 +490,20 @@ bool supported(int G, int k, int Bp) {
 }
 
 size_t step_smem(int Bp, int k, int G) { return v2::step_layout(Bp, k, G).total; }
+cudaError_t tmap_2d(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+                    uint32_t box_inner, uint32_t box_outer);
 template <int kG, int kK, int kUpd>
 cudaError_t launch_step_t(const v2::StepArgs& a, int grid, const void* Xt, const void* W, cudaStream_t st) {
   const size_t smem = step_smem(a.sh.Bp, kK, kG);
   auto kern = v2::k_step2<kG, kK, kUpd>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
+  // the group-major gradient buffer [n_groups * Bp, G] as the stores' tensor: one box per group
+  CUtensorMap tm_dy;
+  e = tmap_2d(&tm_dy, a.dY_out, kG, (uint64_t)a.sh.n_groups * a.sh.Bp, (uint64_t)kG * 2, kG, (uint32_t)a.sh.Bp);
+  if (e != cudaSuccess) return e;
   kern<<<grid, v2::kStepThreads, smem, st>>>(a, static_cast<const __nv_bfloat16*>(Xt),
-                                             static_cast<const __nv_bfloat16*>(W));
+                                             static_cast<const __nv_bfloat16*>(W), tm_dy);
   return cudaGetLastError();
 }
 
