@@ -86,8 +86,8 @@ def algorithmic(wl):
 # kernel from one ncu capture (summaries under profiles/), valid only for the
 # source file it was taken on: (config, timed region) -> (bytes, source digest).
 TRAFFIC = {
-    ("670k", "tail_step"): (643.1e6, "6c87e65aba6e9fd4"),
-    ("670k", "topk_score"): (186.2e6, "a08fbb472ccd8c70"),
+    ("670k", "tail_step"): (647.6e6, "c8e981bb0d4fe169"),
+    ("670k", "tail_dx"): (529.9e6, "697f773de5956a06"),
 }
 # timed region -> (source file under csrc/, kernel name in the ncu summaries)
 KERNELS = {"tail_step": ("tail_v2.cu", "k_step2"), "tail_dx": ("dx_band.cu", "k_dx_band"),
