@@ -163,7 +163,9 @@ DxTiling dx_tiling(const haste_plan_s& p, int Bp, int elem, int sms, int smem_op
     per_chunk = (Bp / 128) * t.n_bands;
   }
   int c = std::max(1, sms / per_chunk);
-  if ((int64_t)c > p.n_groups) c = (int)p.n_groups;
+  // chunks of whole ring items (super-groups of 64 labels) for the band kernel
+  const int64_t units = t.ns > 0 ? tail2::dx_items(p.n_groups, p.G) : p.n_groups;
+  if ((int64_t)c > units) c = (int)units;
   t.n_chunks = c;
   return t;
 }
@@ -183,8 +185,13 @@ TailWs tail_ws(const haste_plan_s& p, int B, int elem, const DxTiling& t) {
   off = align256(off + (size_t)p.d * Bp * elem);
   w.dx_part = off;
   off = align256(off + (size_t)t.n_chunks * p.d * Bp * 4);
-  w.dy_buf = off;  // [B, L] (staged kernels) or group-major [n_groups, Bp, G]
-  off = align256(off + (size_t)Bp * p.n_groups * p.G * elem);
+  // [B, L] (staged kernels) or the fused step's buffer [n_items][Bp][64]: items
+  // of 64 / G groups, whose 64 labels cover the G-wide groups (the last item may
+  // be partial)
+  w.dy_buf = off;
+  size_t dy_elems = (size_t)Bp * p.n_groups * p.G;
+  if (p.G <= 64 && 64 % p.G == 0) dy_elems = std::max(dy_elems, (size_t)tail2::dx_items(p.n_groups, p.G) * Bp * 64);
+  off = align256(off + dy_elems * elem);
   w.loss_part = off;
   off = align256(off + (size_t)kMaxLossParts * 4);
   w.total = off;
@@ -243,7 +250,7 @@ TailArgs make_args(const haste_plan_s& p, int B) {
 }
 
 // dX pass through a pipelined bf16 kernel, from the caller's row-major [B, L]
-// gradient or from the fused step's group-major buffer [n_groups, Bp, G].
+// gradient or from the fused step's buffer [n_groups / (64 / G)][Bp][64].
 cudaError_t dx_v2(const haste_plan_s& p, int B, const void* W, const void* dY, bool group_major, float* part,
                   const DxTiling& t, cudaStream_t s) {
   v2::DxArgs a{};
@@ -257,9 +264,7 @@ cudaError_t dx_v2(const haste_plan_s& p, int B, const void* W, const void* dY, b
   a.n_halves = t.n_halves;
   a.n_chunks = t.n_chunks;
   a.ns = t.ns;
-  // element (b, g*G + j) of dY sits at dY[g*gstride + b*rstride + j]
-  a.dy_gstride = group_major ? (int64_t)a.sh.Bp * p.G : p.G;
-  a.dy_rstride = group_major ? p.G : a.sh.L;
+  a.group_major = group_major ? 1 : 0;
   return tail2::launch_dx(p.G, p.k, a, dY, W, s);
 }
 

@@ -2,12 +2,19 @@
 // (HASTE, "Hardware-Aware Dynamic Sparse Training for Large Output Spaces",
 // Methodology 1; the dX step of the backward pass).
 //
-// k_dx_band -- per CTA (feature band, group chunk, batch half of up to 256 rows): warp 0 loads
-//   each group's dY tile and G x k weight block into a shared-memory ring with
-//   TMA, warps 2-9 (two sets of four, alternate groups) densify the weight block
-//   over the band, warp 1 issues one MMA per 128-row batch tile into TMEM
-//   accumulators, and warps 2-9 write the chunk partial at the end.  k_dx_reduce
-//   (tail.cu) sums the chunk partials in order.
+// k_dx_band -- per CTA (feature band, group chunk, batch half of up to 256 rows):
+//   warp 0 loads each ring item's dY tile and weight rows into a shared-memory
+//   ring with TMA, warps 2-9 (two sets of four, alternate items) densify the
+//   weight rows over the band, warp 1 issues the item's MMAs per 128-row batch
+//   tile into TMEM accumulators, and warps 2-9 write the chunk partial at the end.
+//   k_dx_reduce (tail.cu) sums the chunk partials in order.
+//
+// A ring item is a super-group: NG = 64 / G consecutive groups, 64 labels.  Its
+// dY columns and weight rows are contiguous (row-major dY [B, L], W [L, k]; the
+// fused step writes its gradient buffer as [n_groups / NG][Bp][64]), so one TMA
+// box per operand carries the whole item, with rows of 128 bytes, and one item's
+// MMA chain has K = 64 whatever G: groups of 16 or 32 labels cost the ring round
+// trip of one group of 64.
 
 #include "tail.cuh"
 
@@ -17,31 +24,35 @@ namespace v2 {
 struct DxArgs {
   TailShape sh;
   const int32_t* idx;
-  const __nv_bfloat16* dY;  // for L2 prefetches of the group-major buffer
+  const __nv_bfloat16* dY;  // for L2 prefetches of the fused step's buffer
   const __nv_bfloat16* W;
   float* dX_part;
   int band, n_bands, n_chunks, ns;  // ns: stages of the shared-memory ring
   int n_halves;                      // batch halves of up to 256 rows (2 when B > 256)
-  // element (b, g*G + j) of dY is at dY[g*dy_gstride + b*dy_rstride + j]
-  int64_t dy_gstride, dy_rstride;
-  // dY tile of group g (the batch half's rows) in the dY tensor map: x = g*dy_xg,
-  // y = g*dy_yg + 256*half
-  int dy_xg, dy_yg;
+  int group_major;                   // dY is the fused step's buffer [n_sg][Bp][64], else [B, L]
 };
 
 constexpr int kMaxDxStages = 6;  // deepest ring of the dX pass
-constexpr int kDxPrefetch = 8;   // groups ahead of the ring loads that are prefetched into L2
+constexpr int kDxPrefetch = 8;   // items ahead of the ring loads that are prefetched into L2
+constexpr int kItemLabels = 64;  // labels of a ring item (a super-group)
+
+// Groups per ring item, and the number of items (super-groups) of n_groups groups.
+__host__ __device__ constexpr int items_ng(int G) { return kItemLabels / G; }
+__host__ __device__ inline int64_t n_items_of(int64_t n_groups, int G) {
+  return (n_groups + items_ng(G) - 1) / items_ng(G);
+}
 
 struct DxLayout {
   uint32_t dy, w, wt, bars, total, dy_stride, w_stride, wt_stride;
 };
-// Shared memory of the dX pass: ns stages of (dY tile [Bp][G], weight block
-// [k/64][G][64], densified weight block [band][G]) and the barriers.
-__host__ __device__ inline DxLayout dx_layout(int Bp, int band, int k, int G, int ns) {
+// Shared memory of the dX pass: ns stages of (dY tile [rows][64], weight rows
+// [k/64][64][64], densified weight block [band][64]; 128-byte rows, 128B
+// swizzle) and the barriers.
+__host__ __device__ inline DxLayout dx_layout(int rows, int band, int k, int ns) {
   DxLayout L;
-  L.dy_stride = (uint32_t)((Bp * G * 2 + 1023) & ~1023);
-  L.w_stride = (uint32_t)(((k / 64) * G * 128 + 1023) & ~1023);
-  L.wt_stride = (uint32_t)((band * G * 2 + 1023) & ~1023);
+  L.dy_stride = (uint32_t)((rows * 128 + 1023) & ~1023);
+  L.w_stride = (uint32_t)(((k / 64) * 64 * 128 + 1023) & ~1023);
+  L.wt_stride = (uint32_t)((band * 128 + 1023) & ~1023);
   uint32_t off = 0;
   L.dy = off;
   off += ns * L.dy_stride;
@@ -58,34 +69,37 @@ __host__ __device__ inline DxLayout dx_layout(int Bp, int band, int k, int G, in
 // ========================================================== k_dx_band
 constexpr int kDxThreads = 320;  // producer warp, MMA warp, two sets of 4 densify / epilogue warps
 
-// The dX pass as one dense product per group and feature band.  For a band of
-// NB features [f0, f0+NB), the densified weight block Wt_g[n][j'] (n over the
-// band, j' over the G labels of group g) holds W[g*G + j', s] in the row of the
-// feature f0 + n = idx[g][s] and zeros elsewhere; then
-//   dX[b, f0 + n] = sum over groups g (ascending) of sum_j' dY[b, g*G + j'] Wt_g[n][j'],
-// one tcgen05 MMA per 128-row batch tile and group (M = 128 batch rows, N = NB,
-// K = G), accumulated in TMEM.  A group's slots hold distinct features, so a
-// (b, f) entry receives exactly that group's term dY_g[b, :] . W_g[:, s].
+// The dX pass as one dense product per item and feature band.  For a band of NB
+// features [f0, f0+NB), the densified weight block Wt_u[n][c] (n over the band,
+// c over the item's 64 labels, group j of the item owning columns [jG, jG+G))
+// holds W[g_j*G + c - jG, s] in the row of the feature f0 + n = idx[g_j][s] and
+// zeros elsewhere; then
+//   dX[b, f0 + n] = sum over items u (ascending) of sum_c dY[b, 64u + c] Wt_u[n][c],
+// MMAs per 128-row batch tile (M = 128 batch rows, N = NB, K = 16 per
+// instruction) over the item's present labels, accumulated in TMEM.  A group's
+// slots hold distinct features, so a (b, f) entry receives exactly group g_j's
+// term dY_g[b, :] . W_g[:, s] for every group of the item, in ascending order.
 // One CTA owns a feature band, a batch half of up to 256 rows (up to two 128-row
-// TMEM accumulators of NB columns) and a chunk of groups:
-//   producer (warp 0, one thread): the dY tile (Bp x G, K-major, swizzled rows of
-//     2G bytes) and the G x k weight block into a stage of the ring with TMA;
-//   densify (two sets of four warps, warps 2-5 for the even groups of the chunk,
-//     6-9 for the odd ones; the thread of slot s): clears the Wt row of slot s's
-//     feature in group i - NS (the previous user of the stage, read from the
-//     index array), then, after a barrier of its set, copies column s of the
-//     weight block into the Wt row of the slot's feature when it falls in the
-//     band;
-//   MMA (warp 1): D[t] += dY_g[128t.., :] . Wt_g^T for each batch tile t;
+// TMEM accumulators of NB columns) and a chunk of whole items:
+//   producer (warp 0, one thread): the item's dY tile (the half's rows x 64
+//     labels, K-major) and its weight rows (64 labels x k) into a ring stage;
+//   densify (two sets of four warps, warps 2-5 for the even items of the chunk,
+//     6-9 for the odd ones; the thread of slot s): clears, for each group of the
+//     item NS back (the previous user of the stage), that group's columns of the
+//     Wt row of slot s's feature, then, after a barrier of its set, writes column
+//     s of each present group's weights into its columns of the row of the
+//     slot's feature when it falls in the band;
+//   MMA (warp 1): D[t] += dY_u[128t.., labels] . Wt_u^T for each batch tile t;
 //   epilogue (warps 2-9): the TMEM accumulators to the chunk partial.
-// The warps of a set run the same number of iterations (one per group of the
+// The warps of a set run the same number of iterations (one per item of the
 // set), so its named barrier always matches; a wait that runs out raises the
 // abort flag and the remaining iterations skip their work.
 template <int kG, int kK>
 __global__ void __launch_bounds__(kDxThreads, 1)
     k_dx_band(DxArgs a, const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__ CUtensorMap tm_w) {
   extern __shared__ __align__(1024) uint8_t smem[];
-  constexpr int RB = kG * 2;  // bytes of a K-major row (G bf16)
+  constexpr int NG = items_ng(kG);  // groups per item
+  constexpr int GB = kG * 2;        // bytes of one group's columns in a 128-byte row
   const int NS = a.ns, NB = a.band;
   const TailShape sh = a.sh;
   const int BH = min(sh.Bp, 256);  // rows of the dY box (a batch half)
@@ -95,18 +109,21 @@ __global__ void __launch_bounds__(kDxThreads, 1)
   const int MT = min(2, (sh.Bp - 256 * bh) / 128);  // 128-row tiles of this half
   const int f0 = h * NB;
   const int nf = min(sh.d, f0 + NB) - f0;
-  const int64_t g0 = (int64_t)c * sh.n_groups / a.n_chunks;
-  const int64_t g1 = (int64_t)(c + 1) * sh.n_groups / a.n_chunks;
-  const int n = (int)(g1 - g0);
+  const int64_t n_sg = n_items_of(sh.n_groups, kG);
+  const int64_t u0 = (int64_t)c * n_sg / a.n_chunks;
+  const int64_t u1 = (int64_t)(c + 1) * n_sg / a.n_chunks;
+  const int n = (int)(u1 - u0);  // items of the chunk
+  // groups of item u of the chunk: [(u0 + u) * NG, ... + cnt(u))
+  auto cnt = [&](int u) -> int { return (int)min((int64_t)NG, sh.n_groups - (u0 + u) * NG); };
 
-  const DxLayout Lo = dx_layout(BH, NB, kK, kG, NS);
+  const DxLayout Lo = dx_layout(BH, NB, kK, NS);
   const uint32_t base = align1024(smem_u32(smem));
   uint8_t* gbase = smem + (base - smem_u32(smem));
   auto DYS = [&](int st) -> uint32_t { return base + Lo.dy + st * Lo.dy_stride; };
   auto WS = [&](int st) -> uint32_t { return base + Lo.w + st * Lo.w_stride; };
   auto WT = [&](int st) -> uint32_t { return base + Lo.wt + st * Lo.wt_stride; };
   uint64_t* bars = reinterpret_cast<uint64_t*>(gbase + Lo.bars);
-  uint64_t* full = bars;                      // [NS] dY tile + weight block landed (1 + tx bytes)
+  uint64_t* full = bars;                      // [NS] dY tile + weight rows landed (1 + tx bytes)
   uint64_t* empty = full + kMaxDxStages;      // [NS] both read: MMA commit + 4 densify warps
   uint64_t* wt_full = empty + kMaxDxStages;   // [NS] Wt block written (4 densify warps)
   uint64_t* wt_empty = wt_full + kMaxDxStages;  // [NS] Wt block read by the MMA
@@ -145,27 +162,33 @@ __global__ void __launch_bounds__(kDxThreads, 1)
   if (w == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      const uint32_t bytes = (uint32_t)(BH + kK) * RB;  // dY tile + weight block
-      const bool group_major = a.dy_gstride != kG;
+      const uint32_t bytes = (uint32_t)(BH + kK) * 128;  // dY tile + weight rows (full boxes)
+      const int64_t w_elems = sh.L * kK, ix_elems = sh.n_groups * kK;
       // a ring load from HBM takes longer than the ring's MMA work: the tiles of
-      // later groups are requested into L2 ahead of their ring loads
-      auto prefetch = [&](int64_t g) {
-        if (group_major) prefetch_l2(a.dY + g * a.dy_gstride + (int64_t)256 * bh * kG, (uint32_t)(BH * RB));
-        prefetch_l2(a.W + g * kG * kK, (uint32_t)(kG * kK * 2));
-        prefetch_l2(a.idx + g * kK, (uint32_t)(kK * 4));
+      // later items are requested into L2 ahead of their ring loads (ranges clamped
+      // to the tensors)
+      auto prefetch = [&](int64_t sg) {
+        if (a.group_major)
+          prefetch_l2(a.dY + (sg * sh.Bp + 256 * bh) * kItemLabels, (uint32_t)(min(BH, sh.Bp - 256 * bh) * 128));
+        const int64_t w0 = sg * kItemLabels * kK, i0 = sg * NG * kK;
+        prefetch_l2(a.W + w0, (uint32_t)(min((int64_t)kItemLabels * kK, w_elems - w0) * 2));
+        prefetch_l2(a.idx + i0, (uint32_t)(min((int64_t)NG * kK, ix_elems - i0) * 4));
       };
-      for (int i = 0; i < kDxPrefetch && i < n; ++i) prefetch(g0 + i);
+      for (int i = 0; i < kDxPrefetch && i < n; ++i) prefetch(u0 + i);
       int st = 0, ph = 0, issued = 0;
       for (int i = 0; i < n; ++i) {
-        const int64_t g = g0 + i;
-        if (i + kDxPrefetch < n) prefetch(g + kDxPrefetch);
+        const int64_t sg = u0 + i;
+        if (i + kDxPrefetch < n) prefetch(sg + kDxPrefetch);
         if (!wait_or_abort(&empty[st], ph ^ 1, abort_flag)) break;
         ++issued;
         mbar_arrive_expect_tx(&full[st], bytes);
-        tma_load_2d(DYS(st), &tm_dy, (int)(g * a.dy_xg), (int)(g * a.dy_yg + 256 * bh), &full[st]);
+        if (a.group_major)
+          tma_load_2d(DYS(st), &tm_dy, 0, (int)(sg * sh.Bp + 256 * bh), &full[st]);
+        else
+          tma_load_2d(DYS(st), &tm_dy, (int)(sg * kItemLabels), 256 * bh, &full[st]);
 #pragma unroll
         for (int blk = 0; blk < kK / 64; ++blk)
-          tma_load_2d(WS(st) + (uint32_t)(blk * kG * 128), &tm_w, 64 * blk, (int)(g * kG), &full[st]);
+          tma_load_2d(WS(st) + (uint32_t)(blk * 64 * 128), &tm_w, 64 * blk, (int)(sg * kItemLabels), &full[st]);
         if (++st == NS) {
           st = 0;
           ph ^= 1;
@@ -184,12 +207,11 @@ __global__ void __launch_bounds__(kDxThreads, 1)
       if (!__all_sync(0xffffffffu, wait_or_abort(&wt_full[st], ph, abort_flag))) break;
       tc_fence_after();
       if (lane == 0) {
+        const int nk = cnt(i) * (kG / 16);  // K steps of the item's present labels
         for (int t = 0; t < MT; ++t)
-#pragma unroll
-          for (int kk = 0; kk < kG / 16; ++kk) {
-            const uint64_t ad =
-                make_sdesc(DYS(st) + (uint32_t)(t * 128 * RB + kk * 32), 16, 8 * RB, layout_for_rows(RB));
-            const uint64_t bd = make_sdesc(WT(st) + (uint32_t)(kk * 32), 16, 8 * RB, layout_for_rows(RB));
+          for (int kk = 0; kk < nk; ++kk) {
+            const uint64_t ad = make_sdesc(DYS(st) + (uint32_t)(t * 128 * 128 + kk * 32), 16, 1024, kLayoutSw128);
+            const uint64_t bd = make_sdesc(WT(st) + (uint32_t)(kk * 32), 16, 1024, kLayoutSw128);
             mma_ss<false>(tmem + (uint32_t)(t * 256), ad, bd, idesc, (i > 0 || kk > 0) ? 1u : 0u);
           }
         mma_commit(&empty[st]);
@@ -205,60 +227,80 @@ __global__ void __launch_bounds__(kDxThreads, 1)
     __syncwarp();
   } else {
     // ----------------------------------------------- densify, then epilogue
-    const int set = (w - 2) >> 2;          // groups i = set, set + 2, ...
+    const int set = (w - 2) >> 2;          // items i = set, set + 2, ...
     const int s = (threadIdx.x - 64) & 127;  // this thread's slot
     const bool slot_ok = s < kK;
-    // column s of a weight block: 64-slot block s/64, 16-byte chunk (s%64)/8 of each
-    // 128-byte row (TMA 128-byte swizzle), element s%8
-    const uint32_t wcol = (uint32_t)((s >> 6) * kG * 128 + (s & 7) * 2);
+    // column s of the weight rows: 64-slot block s/64, 16-byte chunk (s%64)/8 of
+    // each 128-byte row (TMA 128-byte swizzle), element s%8
+    const uint32_t wcol = (uint32_t)((s >> 6) * 64 * 128 + (s & 7) * 2);
     const uint32_t wchunk = (uint32_t)((s & 63) >> 3);
-    // the slot's feature in group i of the chunk (-1: no such group or slot)
-    auto feat = [&](int i) -> int { return slot_ok && i >= 0 && i < n ? a.idx[(g0 + i) * kK + s] : -1; };
-    // features of this set's next three groups, and of the groups NS before them
+    // the slot's feature in group j of item i, relative to the band (-1 if absent)
+    auto feat = [&](int i, int j) -> int {
+      if (!slot_ok || i < 0 || i >= n || j >= cnt(i)) return -1;
+      return a.idx[((u0 + i) * NG + j) * kK + s] - f0;
+    };
+    // features of this set's next three items, and of the items NS before them
     // (the previous users of the same ring stages), loaded ahead
-    int fa = feat(set), fb = feat(set + 2), fc = feat(set + 4);
-    int oa = feat(set - NS), ob = feat(set + 2 - NS), oc = feat(set + 4 - NS);
-    // ring position of group i, advanced by two groups per iteration (NS >= 2)
+    int fa[NG], fb[NG], fc[NG], oa[NG], ob[NG], oc[NG];
+#pragma unroll
+    for (int j = 0; j < NG; ++j) {
+      fa[j] = feat(set, j);
+      fb[j] = feat(set + 2, j);
+      fc[j] = feat(set + 4, j);
+      oa[j] = feat(set - NS, j);
+      ob[j] = feat(set + 2 - NS, j);
+      oc[j] = feat(set + 4 - NS, j);
+    }
+    // ring position of item i, advanced by two items per iteration (NS >= 2)
     int st = set;
     uint32_t ph = 0;
     for (int i = set; i < n; i += 2) {
-      const int f = fa - f0, r = oa - f0;
-      const bool act = fa >= 0 && f >= 0 && f < nf;
-      const bool old = oa >= 0 && r >= 0 && r < nf;
-      fa = fb;
-      fb = fc;
-      fc = feat(i + 6);
-      oa = ob;
-      ob = oc;
-      oc = feat(i + 6 - NS);
+      int fcur[NG], fold[NG];
+#pragma unroll
+      for (int j = 0; j < NG; ++j) {
+        fcur[j] = fa[j];
+        fold[j] = oa[j];
+        fa[j] = fb[j];
+        fb[j] = fc[j];
+        fc[j] = feat(i + 6, j);
+        oa[j] = ob[j];
+        ob[j] = oc[j];
+        oc[j] = feat(i + 6 - NS, j);
+      }
       uint8_t* wt = gbase + Lo.wt + st * Lo.wt_stride;
-      // the MMA of group i - NS has read this stage's Wt block: clear its rows
+      // the MMA of item i - NS has read this stage's Wt block: clear its groups' columns
       const bool ok = __all_sync(0xffffffffu, wait_or_abort(&wt_empty[st], ph ^ 1u, abort_flag));
       if (ok) {
-        if (old) {
 #pragma unroll
-          for (int cc = 0; cc < kG / 8; ++cc)
-            *reinterpret_cast<uint4*>(wt + swz_rows((uint32_t)(r * RB + cc * 16), RB)) = make_uint4(0, 0, 0, 0);
-        }
+        for (int j = 0; j < NG; ++j)
+          if (fold[j] >= 0 && fold[j] < nf) {
+#pragma unroll
+            for (int cc = 0; cc < GB / 16; ++cc)
+              *reinterpret_cast<uint4*>(wt + sw128((uint32_t)(fold[j] * 128 + j * GB + cc * 16))) =
+                  make_uint4(0, 0, 0, 0);
+          }
       }
-      // every old row is clear before any new row is written (two slots of
-      // different groups may share a feature)
+      // every old column run is clear before any new one is written (slots of
+      // different items may share a feature)
       named_bar(1 + set, 128);
       const bool ok2 = ok && __all_sync(0xffffffffu, wait_or_abort(&full[st], ph, abort_flag));
       if (ok2) {
-        if (act) {
-          const uint8_t* col = gbase + Lo.w + st * Lo.w_stride + wcol;
+        const uint8_t* wst = gbase + Lo.w + st * Lo.w_stride + wcol;
+#pragma unroll
+        for (int j = 0; j < NG; ++j) {
+          const int f = fcur[j];
+          if (f < 0 || f >= nf) continue;
           uint32_t pk[kG / 2];
 #pragma unroll
           for (int l = 0; l < kG; l += 2) {
-            const uint32_t lo = *reinterpret_cast<const uint16_t*>(col + l * 128 + ((wchunk ^ (l & 7)) << 4));
-            const uint32_t hi =
-                *reinterpret_cast<const uint16_t*>(col + (l + 1) * 128 + ((wchunk ^ ((l + 1) & 7)) << 4));
+            const int r0 = j * kG + l, r1 = r0 + 1;  // weight rows (labels) of the item
+            const uint32_t lo = *reinterpret_cast<const uint16_t*>(wst + r0 * 128 + ((wchunk ^ (r0 & 7)) << 4));
+            const uint32_t hi = *reinterpret_cast<const uint16_t*>(wst + r1 * 128 + ((wchunk ^ (r1 & 7)) << 4));
             pk[l / 2] = lo | (hi << 16);
           }
 #pragma unroll
-          for (int cc = 0; cc < kG / 8; ++cc)
-            *reinterpret_cast<uint4*>(wt + swz_rows((uint32_t)(f * RB + cc * 16), RB)) =
+          for (int cc = 0; cc < GB / 16; ++cc)
+            *reinterpret_cast<uint4*>(wt + sw128((uint32_t)(f * 128 + j * GB + cc * 16))) =
                 make_uint4(pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
         }
         fence_proxy_async_smem();
@@ -307,23 +349,24 @@ __global__ void __launch_bounds__(kDxThreads, 1)
 // ------------------------------------------------------------- host side
 namespace tail2 {
 
-size_t dx_smem(int Bp, int band, int k, int G, int ns) { return v2::dx_layout(Bp, band, k, G, ns).total; }
+bool dx_supported(int G, int k, int Bp) {
+  return (G == 16 || G == 32 || G == 64) && (k == 64 || k == 128) && Bp <= 512;
+}
+
+size_t dx_smem(int rows, int band, int k, int ns) { return v2::dx_layout(rows, band, k, ns).total; }
 
 // Feature bands and ring depth of the dX pass: bands of at most 256 features
 // (the widest MMA N), as few as cover d, split evenly in multiples of 16; the
 // deepest ring (up to six stages) that fits in the shared memory left after
 // `reserve` bytes.  Returns false when two stages do not fit.
-bool dx_supported(int G, int k, int Bp) {
-  return (G == 16 || G == 32 || G == 64) && (k == 64 || k == 128) && Bp <= 512;
-}
-
 bool dx_config(int G, int k, int d, int Bp, size_t smem_optin, size_t reserve, int* band, int* n_bands, int* ns) {
-  Bp = Bp < 256 ? Bp : 256;  // a CTA covers a batch half of up to 256 rows
+  (void)G;
+  const int rows = Bp < 256 ? Bp : 256;  // a CTA covers a batch half of up to 256 rows
   const int nb = (d + 255) / 256;
   const int bw = (((d + nb - 1) / nb) + 15) & ~15;
   int best = 0;
   for (int st = 2; st <= v2::kMaxDxStages; ++st)
-    if (dx_smem(Bp, bw, k, G, st) + reserve <= smem_optin) best = st;
+    if (dx_smem(rows, bw, k, st) + reserve <= smem_optin) best = st;
   if (!best) return false;
   *band = bw;
   *n_bands = nb;
@@ -331,29 +374,27 @@ bool dx_config(int G, int k, int d, int Bp, size_t smem_optin, size_t reserve, i
   return true;
 }
 
-// dY of the dX pass, either the group-major buffer [n_groups, Bp, G] of the fused
-// step (dy_gstride = Bp*G, dy_rstride = G; rows past B hold zeros) or a caller's
-// row-major [B, L] (dy_gstride = G, dy_rstride = L; rows past B are outside the
+// Items (super-groups of 64 labels) of the dX pass for n_groups groups of G.
+int64_t dx_items(int64_t n_groups, int G) { return v2::n_items_of(n_groups, G); }
+
+// dY of the dX pass, either the fused step's buffer [n_items][Bp][64] (rows past
+// B hold zeros) or a caller's row-major [B, L] (rows past B are outside the
 // tensor and read as zeros).
 template <int kG, int kK>
 cudaError_t launch_dx_t(v2::DxArgs a, const void* dY, const void* W, cudaStream_t st) {
-  const int BH = a.sh.Bp < 256 ? a.sh.Bp : 256;
-  const size_t smem = dx_smem(BH, a.band, kK, kG, a.ns);
+  const int rows = a.sh.Bp < 256 ? a.sh.Bp : 256;
+  const size_t smem = dx_smem(rows, a.band, kK, a.ns);
   auto kern = v2::k_dx_band<kG, kK>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   CUtensorMap tm_dy, tm_w;
-  const bool group_major = a.dy_gstride != kG;  // row-major [B, L] has dy_gstride = G
-  if (group_major) {
-    e = tmap_2d(&tm_dy, dY, kG, (uint64_t)a.sh.n_groups * a.sh.Bp, (uint64_t)kG * 2, kG, (uint32_t)BH);
-    a.dy_xg = 0;
-    a.dy_yg = a.sh.Bp;
-  } else {
-    e = tmap_2d(&tm_dy, dY, (uint64_t)a.sh.L, (uint64_t)a.sh.B, (uint64_t)a.dy_rstride * 2, kG, (uint32_t)BH);
-    a.dy_xg = kG;
-    a.dy_yg = 0;
-  }
-  if (e == cudaSuccess) e = tmap_2d(&tm_w, W, kK, (uint64_t)a.sh.L, (uint64_t)kK * 2, 64, kG);
+  if (a.group_major)
+    e = tmap_2d(&tm_dy, dY, v2::kItemLabels, (uint64_t)dx_items(a.sh.n_groups, kG) * a.sh.Bp, 128,
+                v2::kItemLabels, (uint32_t)rows);
+  else
+    e = tmap_2d(&tm_dy, dY, (uint64_t)a.sh.L, (uint64_t)a.sh.B, (uint64_t)a.sh.L * 2, v2::kItemLabels,
+                (uint32_t)rows);
+  if (e == cudaSuccess) e = tmap_2d(&tm_w, W, kK, (uint64_t)a.sh.L, (uint64_t)kK * 2, 64, v2::kItemLabels);
   if (e != cudaSuccess) return e;
   const int grid = a.n_bands * a.n_halves * a.n_chunks;
   kern<<<grid, v2::kDxThreads, smem, st>>>(a, tm_dy, tm_w);

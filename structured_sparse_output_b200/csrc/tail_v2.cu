@@ -11,8 +11,8 @@
 //              while the epilogue runs;
 //   warps 5-12 epilogue: logits leave TMEM only as the BCE gradient (bf16, into
 //              shared memory: the dW operand, and the tile that the MMA thread
-//              writes to the group-major gradient buffer of the dX pass with one
-//              TMA store); the BCE of group i+1 comes before the dW readout of
+//              writes to the gradient buffer of the dX pass with one TMA store,
+//              items of 64 / G groups side by side in 128-byte rows); the BCE of group i+1 comes before the dW readout of
 //              group i, so the dW product runs behind it.  The readout
 //              writes dW, or (kUpd > 0) applies an SGD update to the group's
 //              weights while dW is on chip: M' = momentum * M + dW (kUpd = 2) or
@@ -33,7 +33,7 @@ struct StepArgs {
   __nv_bfloat16* W_out;   // kUpd > 0: updated weights [L, k]
   __nv_bfloat16* M;       // kUpd = 2: momentum [L, k], updated in place
   float lr, momentum;
-  __nv_bfloat16* dY_out;  // group-major gradient buffer [n_groups, Bp, G]
+  __nv_bfloat16* dY_out;  // gradient buffer [n_groups / (64 / G)][Bp][64] of the dX pass
   float* loss_part;
   const int32_t* pos_ptr;
   const int32_t* pos_ids;
@@ -259,8 +259,13 @@ __global__ void __launch_bounds__(kStepThreads, 1)
             }
             mma_commit(&dw_full[s]);
             mma_commit(&empty[s]);
-            // the group's gradient tile to the dX pass's group-major buffer
-            tma_store_2d(&tm_dy, base + DY(s), 0, (int)((gb + nd) * Bp));
+            // the group's gradient tile to the dX pass's buffer: columns of its
+            // item (64 / G consecutive groups, 64 labels), the item's Bp rows
+            {
+              const int64_t g = gb + nd;
+              constexpr int NG = 64 / kG;
+              tma_store_2d(&tm_dy, base + DY(s), (int)(g % NG) * kG, (int)((g / NG) * Bp));
+            }
             bulk_commit();
           }
           __syncwarp();
@@ -498,9 +503,11 @@ cudaError_t launch_step_t(const v2::StepArgs& a, int grid, const void* Xt, const
   auto kern = v2::k_step2<kG, kK, kUpd>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  // the group-major gradient buffer [n_groups * Bp, G] as the stores' tensor: one box per group
+  // the gradient buffer [n_items * Bp][64] as the stores' tensor: group g's box
+  // (G labels x Bp rows) at columns (g % NG) * G of item g / NG's rows, NG = 64 / G
   CUtensorMap tm_dy;
-  e = tmap_2d(&tm_dy, a.dY_out, kG, (uint64_t)a.sh.n_groups * a.sh.Bp, (uint64_t)kG * 2, kG, (uint32_t)a.sh.Bp);
+  const uint64_t n_items = (uint64_t)(a.sh.n_groups + 64 / kG - 1) / (64 / kG);
+  e = tmap_2d(&tm_dy, a.dY_out, 64, n_items * a.sh.Bp, 128, kG, (uint32_t)a.sh.Bp);
   if (e != cudaSuccess) return e;
   kern<<<grid, v2::kStepThreads, smem, st>>>(a, static_cast<const __nv_bfloat16*>(Xt),
                                              static_cast<const __nv_bfloat16*>(W), tm_dy);
