@@ -185,7 +185,7 @@ TailWs tail_ws(const haste_plan_s& p, int B, int elem, const DxTiling& t) {
   off = align256(off + (size_t)p.d * Bp * elem);
   w.dx_part = off;
   off = align256(off + (size_t)t.n_chunks * p.d * Bp * 4);
-  // [B, L] (staged kernels) or the fused step's buffer [n_items][Bp][64]: items
+  // [B, L] (staged kernels) or the fused step's buffer [n_items * 64][Bp]: items
   // of 64 / G groups, whose 64 labels cover the G-wide groups (the last item may
   // be partial)
   w.dy_buf = off;
@@ -250,7 +250,7 @@ TailArgs make_args(const haste_plan_s& p, int B) {
 }
 
 // dX pass through a pipelined bf16 kernel, from the caller's row-major [B, L]
-// gradient or from the fused step's buffer [n_groups / (64 / G)][Bp][64].
+// gradient or from the fused step's buffer of label rows [n_items * 64][Bp].
 cudaError_t dx_v2(const haste_plan_s& p, int B, const void* W, const void* dY, bool group_major, float* part,
                   const DxTiling& t, cudaStream_t s) {
   v2::DxArgs a{};

@@ -68,6 +68,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// Non-blocking test of the phase with the given parity (mbarrier.test_wait never
+// suspends the thread, unlike try_wait): for threads that poll several barriers.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
 // As mbar_try_wait, but a thread whose phase is not complete yet is suspended
 // (it issues nothing) until the phase completes or about hint_ns pass.
 __device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
@@ -144,6 +157,18 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32
 __device__ __forceinline__ void named_bar(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
+// Named barrier that also ORs a predicate over its threads: every thread gets the
+// same answer.
+__device__ __forceinline__ bool named_bar_or(int id, int nthreads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred c, p;\n\tsetp.ne.u32 c, %2, 0;\n\tbar.red.or.pred p, %1, %3, c;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r)
+      : "r"(id), "r"((uint32_t)pred), "r"(nthreads)
+      : "memory");
+  return r != 0;
+}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 // Make generic-proxy shared-memory writes visible to the tensor core (async proxy).
@@ -216,6 +241,21 @@ __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
   }
+}
+// Weight-stationary form, cta_group::1 (tcgen05.mma.ws): M in {32, 64, 128}, N in
+// {64, 128, 256}.  Where D sits in TMEM (N columns of fp32 in total):
+//   M = 32: row m in lane 32q + m of every lane quarter q, which holds the
+//           columns n in [qN/4, (q+1)N/4) at column offset n - qN/4;
+//   M = 64: rows 0-63 in lanes 0-63 for n < N/2 and in lanes 64-127 for
+//           n >= N/2, at column offset n mod N/2.
+// For a small M the instruction costs far less than a 128-row one of the same N.
+__device__ __forceinline__ void mma_ws(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                       uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.ws.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
 }
 // Arrive once on the mbarrier when all previously issued MMAs of this thread finish.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {

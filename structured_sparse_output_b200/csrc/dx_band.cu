@@ -11,10 +11,10 @@
 //
 // A ring item is a super-group: NG = 64 / G consecutive groups, 64 labels.  Its
 // dY columns and weight rows are contiguous (row-major dY [B, L], W [L, k]; the
-// fused step writes its gradient buffer as [n_groups / NG][Bp][64]), so one TMA
-// box per operand carries the whole item, with rows of 128 bytes, and one item's
-// MMA chain has K = 64 whatever G: groups of 16 or 32 labels cost the ring round
-// trip of one group of 64.
+// fused step writes its gradient buffer transposed, as label rows [n_items * 64]
+// [Bp]), so a few TMA boxes per operand carry the whole item, with rows of 128
+// bytes, and one item's MMA chain has K = 64 whatever G: groups of 16 or 32
+// labels cost the ring round trip of one group of 64.
 
 #include "tail.cuh"
 
@@ -29,7 +29,7 @@ struct DxArgs {
   float* dX_part;
   int band, n_bands, n_chunks, ns;  // ns: stages of the shared-memory ring
   int n_halves;                      // batch halves of up to 256 rows (2 when B > 256)
-  int group_major;                   // dY is the fused step's buffer [n_sg][Bp][64], else [B, L]
+  int group_major;                   // dY is the fused step's buffer [n_items * 64][Bp], else [B, L]
 };
 
 constexpr int kMaxDxStages = 6;  // deepest ring of the dX pass
@@ -168,8 +168,7 @@ __global__ void __launch_bounds__(kDxThreads, 1)
       // later items are requested into L2 ahead of their ring loads (ranges clamped
       // to the tensors)
       auto prefetch = [&](int64_t sg) {
-        if (a.group_major)
-          prefetch_l2(a.dY + (sg * sh.Bp + 256 * bh) * kItemLabels, (uint32_t)(min(BH, sh.Bp - 256 * bh) * 128));
+        if (a.group_major) prefetch_l2(a.dY + sg * kItemLabels * sh.Bp, (uint32_t)(kItemLabels * sh.Bp * 2));
         const int64_t w0 = sg * kItemLabels * kK, i0 = sg * NG * kK;
         prefetch_l2(a.W + w0, (uint32_t)(min((int64_t)kItemLabels * kK, w_elems - w0) * 2));
         prefetch_l2(a.idx + i0, (uint32_t)(min((int64_t)NG * kK, ix_elems - i0) * 4));
@@ -182,9 +181,11 @@ __global__ void __launch_bounds__(kDxThreads, 1)
         if (!wait_or_abort(&empty[st], ph ^ 1, abort_flag)) break;
         ++issued;
         mbar_arrive_expect_tx(&full[st], bytes);
-        if (a.group_major)
-          tma_load_2d(DYS(st), &tm_dy, 0, (int)(sg * sh.Bp + 256 * bh), &full[st]);
-        else
+        if (a.group_major) {
+          for (int blk = 0; blk < BH / 64; ++blk)
+            tma_load_2d(DYS(st) + (uint32_t)(blk * 64 * 128), &tm_dy, 256 * bh + 64 * blk, (int)(sg * kItemLabels),
+                        &full[st]);
+        } else
           tma_load_2d(DYS(st), &tm_dy, (int)(sg * kItemLabels), 256 * bh, &full[st]);
 #pragma unroll
         for (int blk = 0; blk < kK / 64; ++blk)
@@ -200,7 +201,7 @@ __global__ void __launch_bounds__(kDxThreads, 1)
     }
   } else if (w == 1) {
     // ------------------------------------------------------------- MMA
-    const uint32_t idesc = make_idesc(1, 0, 0, 128, (uint32_t)NB);
+    const uint32_t idesc = make_idesc(1, a.group_major ? 1u : 0u, 0, 128, (uint32_t)NB);
     int st = 0, ph = 0;
     for (int i = 0; i < n; ++i) {
       if (!__all_sync(0xffffffffu, wait_or_abort(&full[st], ph, abort_flag))) break;
@@ -210,7 +211,12 @@ __global__ void __launch_bounds__(kDxThreads, 1)
         const int nk = cnt(i) * (kG / 16);  // K steps of the item's present labels
         for (int t = 0; t < MT; ++t)
           for (int kk = 0; kk < nk; ++kk) {
-            const uint64_t ad = make_sdesc(DYS(st) + (uint32_t)(t * 128 * 128 + kk * 32), 16, 1024, kLayoutSw128);
+            // the fused step's tile is label rows (batch contiguous: MN-major, 64-row
+            // blocks 8 KB apart), a caller's is batch rows (labels contiguous: K-major)
+            const uint64_t ad =
+                a.group_major
+                    ? make_sdesc(DYS(st) + (uint32_t)(t * 2 * 64 * 128 + kk * 16 * 128), 64 * 128, 1024, kLayoutSw128)
+                    : make_sdesc(DYS(st) + (uint32_t)(t * 128 * 128 + kk * 32), 16, 1024, kLayoutSw128);
             const uint64_t bd = make_sdesc(WT(st) + (uint32_t)(kk * 32), 16, 1024, kLayoutSw128);
             mma_ss<false>(tmem + (uint32_t)(t * 256), ad, bd, idesc, (i > 0 || kk > 0) ? 1u : 0u);
           }
@@ -377,9 +383,9 @@ bool dx_config(int G, int k, int d, int Bp, size_t smem_optin, size_t reserve, i
 // Items (super-groups of 64 labels) of the dX pass for n_groups groups of G.
 int64_t dx_items(int64_t n_groups, int G) { return v2::n_items_of(n_groups, G); }
 
-// dY of the dX pass, either the fused step's buffer [n_items][Bp][64] (rows past
-// B hold zeros) or a caller's row-major [B, L] (rows past B are outside the
-// tensor and read as zeros).
+// dY of the dX pass, either the fused step's buffer of label rows [n_items * 64]
+// [Bp] (columns past B hold zeros) or a caller's row-major [B, L] (rows past B are
+// outside the tensor and read as zeros).
 template <int kG, int kK>
 cudaError_t launch_dx_t(v2::DxArgs a, const void* dY, const void* W, cudaStream_t st) {
   const int rows = a.sh.Bp < 256 ? a.sh.Bp : 256;
@@ -389,8 +395,8 @@ cudaError_t launch_dx_t(v2::DxArgs a, const void* dY, const void* W, cudaStream_
   if (e != cudaSuccess) return e;
   CUtensorMap tm_dy, tm_w;
   if (a.group_major)
-    e = tmap_2d(&tm_dy, dY, v2::kItemLabels, (uint64_t)dx_items(a.sh.n_groups, kG) * a.sh.Bp, 128,
-                v2::kItemLabels, (uint32_t)rows);
+    e = tmap_2d(&tm_dy, dY, (uint64_t)a.sh.Bp, (uint64_t)dx_items(a.sh.n_groups, kG) * v2::kItemLabels,
+                (uint64_t)a.sh.Bp * 2, 64, v2::kItemLabels);
   else
     e = tmap_2d(&tm_dy, dY, (uint64_t)a.sh.L, (uint64_t)a.sh.B, (uint64_t)a.sh.L * 2, v2::kItemLabels,
                 (uint32_t)rows);

@@ -2,22 +2,30 @@
 // tail (HASTE, "Hardware-Aware Dynamic Sparse Training for Large Output Spaces",
 // Methodology 1: labels in groups of G share one fan-in set I_g of k features).
 //
-// k_step2 -- fused forward + BCE gradient + dW, one group per iteration:
-//   warps 0-3  producers: the gather-once tile X[:, I_g] (k rows of X^T) and the
-//              G x k weight block, staged with cp.async into a 2-stage ring; warps
-//              0 and 2 fill stage 0, warps 1 and 3 stage 1;
+// k_step2 -- fused forward + BCE gradient + dW, one group per iteration, with the
+// group's labels as the small M of weight-stationary MMAs (MW = 32 rows for G <= 32,
+// 64 for G = 64), so that one instruction covers the whole batch (forward: N = Bp)
+// or every slot (dW: N = k):
+//   forward  logits_g^T [MW, Bp] = W_g [MW, k] . Xg^T     (K = k)
+//   dW       dW_g^T     [MW, k]  = dY_g^T [MW, Bp] . Xg   (K = Bp)
+//   warps 0-3  producers: the gather-once tile Xg = X[:, I_g] (k rows of X^T) and
+//              the G x k weight block, staged with cp.async into a 2-stage ring
+//              (all four warps fill the stage of each group);
 //   warp 4     MMA issuer (one thread): issues each group's forward and dW
-//              product as soon as its inputs are ready, so the tensor core works
-//              while the epilogue runs;
-//   warps 5-12 epilogue: logits leave TMEM only as the BCE gradient (bf16, into
-//              shared memory: the dW operand, and the tile that the MMA thread
-//              writes to the gradient buffer of the dX pass with one TMA store,
-//              items of 64 / G groups side by side in 128-byte rows); the BCE of group i+1 comes before the dW readout of
-//              group i, so the dW product runs behind it.  The readout
-//              writes dW, or (kUpd > 0) applies an SGD update to the group's
-//              weights while dW is on chip: M' = momentum * M + dW (kUpd = 2) or
-//              M' = dW (kUpd = 1), W' = W - lr * M', with W' written to a
-//              separate buffer (the dX pass still reads W) and M' over M.
+//              product as soon as its inputs are ready;
+//   warps 5-12 epilogue: each thread owns one label and a run of batch rows of the
+//              logits; they leave TMEM only as the BCE gradient dY^T (bf16, into
+//              shared memory: the dW operand, and the tile that epilogue thread 0
+//              writes to the gradient buffer of the dX pass with TMA stores).  The
+//              positives of the group come from a per-row cursor over the sorted
+//              CSR targets, turned into label x row bit masks in shared memory.
+//              The BCE of group i+1 comes before the dW readout of group i, so the
+//              dW product runs behind it.  The readout writes dW as 16-byte
+//              vectors (one label row, consecutive slots), or (kUpd > 0) applies an
+//              SGD update to the group's weights while dW is on chip:
+//              M' = momentum * M + dW (kUpd = 2) or M' = dW (kUpd = 1),
+//              W' = W - lr * M', with W' written to a separate buffer (the dX pass
+//              still reads W) and M' over M.
 //
 // The dX pass that reads the gradient buffer is in dx_band.cu.
 
@@ -33,26 +41,34 @@ struct StepArgs {
   __nv_bfloat16* W_out;   // kUpd > 0: updated weights [L, k]
   __nv_bfloat16* M;       // kUpd = 2: momentum [L, k], updated in place
   float lr, momentum;
-  __nv_bfloat16* dY_out;  // gradient buffer [n_groups / (64 / G)][Bp][64] of the dX pass
+  __nv_bfloat16* dY_out;  // gradient buffer of the dX pass: [n_items * 64][Bp], label rows
   float* loss_part;
   const int32_t* pos_ptr;
   const int32_t* pos_ids;
   float grad_scale;
 };
 
+// Rows of the weight-stationary MMAs for groups of G labels.
+__host__ __device__ constexpr int step_mw(int G) { return G <= 32 ? 32 : 64; }
+
 // ------------------------------------------------------------ smem layouts
+// Per stage: Xg [Bp/64][k][64] (slot rows, 64 batch columns per 128-byte row),
+// W_g [k/64][MW][64] (label rows, 64 slots per row) and dY^T [Bp/64][MW][64]
+// (label rows, 64 batch columns per row), all 128B-swizzled.  After the forward
+// has read W_g, its space holds the group's positive-label bit masks.
 struct StepLayout {
   uint32_t xg[2], wg[2], dy[2], bars, total;
 };
 __host__ __device__ inline StepLayout step_layout(int Bp, int k, int G) {
   StepLayout L;
-  const uint32_t xg = (uint32_t)((Bp / 64) * k * 128 + (k < 128 ? (128 - k) * 128 : 0));
-  const uint32_t wg = (uint32_t)((k / 64) * G * 128);
-  const uint32_t dy = (uint32_t)(Bp * G * 2);
+  const int MW = step_mw(G);
+  const uint32_t xg = (uint32_t)((Bp / 64) * k * 128);
+  const uint32_t wg = (uint32_t)((k / 64) * MW * 128);
+  const uint32_t dy = (uint32_t)((Bp / 64) * MW * 128);
   uint32_t off = 0;
   for (int s = 0; s < 2; ++s) { L.xg[s] = off; off += xg; }
   for (int s = 0; s < 2; ++s) { L.wg[s] = off; off += wg; }
-  for (int s = 0; s < 2; ++s) { L.dy[s] = off; off += (dy + 1023u) & ~1023u; }
+  for (int s = 0; s < 2; ++s) { L.dy[s] = off; off += dy; }
   L.bars = off;
   off += 256;
   L.total = off + 1024;
@@ -80,23 +96,29 @@ __device__ __forceinline__ void publish_all(uint64_t* full_bar) {
   mbar_arrive(full_bar);
 }
 
+// 32 lanes x 32 consecutive 32-bit TMEM columns (two x16 loads; one wait after).
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
+  tmem_ld16(taddr, *reinterpret_cast<float(*)[16]>(v));
+  tmem_ld16(taddr + 16, *reinterpret_cast<float(*)[16]>(v + 16));
+}
+
 // ============================================================ k_step2
 constexpr int kStepProd = 4;       // producer warps: two per ring stage
 constexpr int kStepMma = kStepProd;  // warp id of the MMA issuer
 constexpr int kStepEpi = 8;        // epilogue warps: 4 lane quarters x 2 column halves
 constexpr int kStepThreads = 32 * (kStepProd + 1 + kStepEpi);  // producers, MMA warp, epilogue warps
-constexpr int kMaxPosReg = 8;      // positives per batch row kept in registers
+constexpr int kStepEpiThreads = 32 * kStepEpi;
 
 template <int kG, int kK, int kUpd>
 __global__ void __launch_bounds__(kStepThreads, 1)
     k_step2(StepArgs a, const __nv_bfloat16* __restrict__ Xt, const __nv_bfloat16* __restrict__ W,
             const __grid_constant__ CUtensorMap tm_dy) {
   extern __shared__ __align__(1024) uint8_t smem[];
-  constexpr int RB = kG * 2;   // bytes of one dY row in shared memory
-  constexpr int CH = kG / 2;   // label columns per epilogue half
+  constexpr int MW = step_mw(kG);     // rows of the weight-stationary MMAs
+  constexpr int NGI = 64 / kG;        // groups per 64-label item of the gradient buffer
   constexpr int kRowsPerThr = kK / 4;
   const TailShape sh = a.sh;
-  const int Bp = sh.Bp, n_bt = Bp / 128;
+  const int Bp = sh.Bp;
   const StepLayout Lo = step_layout(Bp, kK, kG);
   const uint32_t base = align1024(smem_u32(smem));
   uint8_t* gbase = smem + (base - smem_u32(smem));
@@ -115,7 +137,7 @@ __global__ void __launch_bounds__(kStepThreads, 1)
   const int w = warp_id(), lane = lane_id();
   if (threadIdx.x == 0) {
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&full[s], 32 * kStepProd / 2);
+      mbar_init(&full[s], 32 * kStepProd);
       mbar_init(&empty[s], 1);
       mbar_init(&fwd_full[s], 1);
       mbar_init(&dy_full[s], kStepEpi);
@@ -126,9 +148,11 @@ __global__ void __launch_bounds__(kStepThreads, 1)
     *abort_flag = 0;
     fence_mbar_init();
   }
-  // TMEM: forward accumulators F[2] (n_bt*G columns each), dW accumulators D[2]
-  const uint32_t f_cols = (uint32_t)(n_bt * kG);
-  const uint32_t ncols = tmem_cols_for(2 * f_cols + 2 * kG);
+  // TMEM: logits^T accumulators F[2] (Bp columns over the lane quarters: Bp/4 for
+  // MW = 32, Bp/2 for MW = 64), dW^T accumulators D[2] (k/4 or k/2 columns)
+  const uint32_t f_cols = (uint32_t)(MW == 32 ? Bp / 4 : Bp / 2);
+  constexpr uint32_t d_cols = MW == 32 ? kK / 4 : kK / 2;
+  const uint32_t ncols = tmem_cols_for(2 * f_cols + 2 * d_cols);
   if (w == kStepMma) {
     tmem_alloc(tslot, ncols);
     tmem_relinquish();
@@ -138,7 +162,7 @@ __global__ void __launch_bounds__(kStepThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tslot;
   auto F = [&](int s) -> uint32_t { return tmem + (s ? f_cols : 0u); };
-  auto D = [&](int s) -> uint32_t { return tmem + 2 * f_cols + (s ? (uint32_t)kG : 0u); };
+  auto D = [&](int s) -> uint32_t { return tmem + 2 * f_cols + (s ? d_cols : 0u); };
   auto XG = [&](int s) -> uint32_t { return base + (s ? Lo.xg[1] : Lo.xg[0]); };
   auto WG = [&](int s) -> uint32_t { return base + (s ? Lo.wg[1] : Lo.wg[0]); };
   auto DY = [&](int s) -> uint32_t { return s ? Lo.dy[1] : Lo.dy[0]; };
@@ -150,20 +174,19 @@ __global__ void __launch_bounds__(kStepThreads, 1)
 
   if (w < kStepProd) {
     // ------------------------------------------------- cp.async producers
-    // warps (half, part) fill stage half with the items i = half, half+2, ...;
-    // each of the two warps of a stage copies every other group of four rows.
-    // Lane (rg, sub) copies the 16-byte chunk sub of every 128-byte segment of
-    // its rows, so that 8 consecutive lanes read one segment; the feature
-    // indices of its rows sit in registers.
-    constexpr int P = kStepProd / 2;
+    // all four warps fill the stage of every item i (stage i & 1); warp part
+    // copies every fourth group of four rows.  Lane (rg, sub) copies the 16-byte
+    // chunk sub of every 128-byte segment of its rows, so that 8 consecutive lanes
+    // read one segment; the feature indices of its rows sit in registers.
+    constexpr int P = kStepProd;
     constexpr int kRows = kRowsPerThr / P;
-    const int half = w & 1, part = w >> 1, ht = lane;
+    const int part = w, ht = lane;
     const int sub = ht & 7, rg = ht >> 3;
-    const uint32_t xg = XG(half), wg = WG(half);
-    int i = half;
-    for (; i < n_items; i += 2) {
+    for (int i = 0; i < n_items; ++i) {
       const int64_t g = gb + i;
-      // this half's next group: weight block and indices into L2 (from HBM they
+      const int half = i & 1;
+      const uint32_t xg = XG(half), wg = WG(half);
+      // the group after next: weight block and indices into L2 (from HBM they
       // would stretch the gather of that group)
       if (part == 0 && lane == 0 && i + 2 < n_items) {
         prefetch_l2(W + (g + 2) * kG * kK, (uint32_t)(kG * kK * 2));
@@ -185,14 +208,15 @@ __global__ void __launch_bounds__(kStepThreads, 1)
         for (int bb = 0; bb < 4; ++bb)
           if (bb < nbb) cp_async16(dst + (uint32_t)(bb * kK * 128), src + bb * 64, 16);
       }
-      // weight block of the group (contiguous G x k), chunks split between the warps
+      // weight block of the group (contiguous G x k) into label rows of MW-row
+      // blocks of 64 slots; chunks split between the warps
       const __nv_bfloat16* wsrc = W + g * (int64_t)kG * kK;
       constexpr int cpr = kK / 8;
 #pragma unroll 4
       for (int c0 = 32 * part; c0 < kG * cpr; c0 += 32 * P) {
         const int c = c0 + ht;
         const int j = c / cpr, cc = c % cpr;
-        cp_async16(wg + sw128((uint32_t)((cc >> 3) * kG * 128 + j * 128 + (cc & 7) * 16)),
+        cp_async16(wg + sw128((uint32_t)((cc >> 3) * MW * 128 + j * 128 + (cc & 7) * 16)),
                    wsrc + (int64_t)j * kK + cc * 8, 16);
       }
       cp_async_commit();
@@ -207,8 +231,12 @@ __global__ void __launch_bounds__(kStepThreads, 1)
     // dW(j) needs the BCE of j (dy_full) and D(j&1) read out for j-2
     // (tmem_empty).  Lane 0 polls; the decisions are broadcast so the warp stays
     // converged.  No progress for the wait limit raises the abort flag.
-    const uint32_t idesc_f = make_idesc(1, 1, 0, 128, kG);
-    const uint32_t idesc_w = make_idesc(1, 0, 1, 128, kG);
+    //   forward: A = W_g (K-major, label rows), B = Xg (MN-major: batch
+    //            contiguous, 64-column blocks kK*128 bytes apart), K = 16 slots;
+    //   dW:      A = dY^T (K-major, label rows), B = Xg (K-major: slot rows),
+    //            K = 16 batch rows.
+    const uint32_t idesc_f = make_idesc(1, 0, 1, MW, (uint32_t)Bp);
+    const uint32_t idesc_w = make_idesc(1, 0, 0, MW, kK);
     int nf = 0, nd = 0;
     uint64_t t_last = globaltimer_ns();
     const uint64_t limit = g_wait_limit_ns;
@@ -217,22 +245,17 @@ __global__ void __launch_bounds__(kStepThreads, 1)
       bool did = false;
       if (nf < n_items && nf <= nd + 1) {
         const int s = nf & 1;
-        const bool rdy = __shfl_sync(0xffffffffu, lane == 0 ? mbar_try_wait(&full[s], (nf >> 1) & 1) : false, 0);
+        const bool rdy = __shfl_sync(0xffffffffu, lane == 0 ? mbar_test_wait(&full[s], (nf >> 1) & 1) : false, 0);
         if (rdy) {
           if (lane == 0) {
             tc_fence_after();
-            for (int t = 0; t < n_bt; ++t)
-              for (int kk = 0; kk < kK / 16; ++kk) {
-                const uint64_t ad = make_sdesc(XG(s) + (uint32_t)(t * 2 * kK * 128 + kk * 16 * 128),
-                                               (uint32_t)kK * 128, 1024, kLayoutSw128);
-                const uint64_t bd =
-                    make_sdesc(WG(s) + (uint32_t)((kk / 4) * kG * 128 + (kk % 4) * 32), 16, 1024, kLayoutSw128);
-                mma_ss<false>(F(s) + (uint32_t)(t * kG), ad, bd, idesc_f, kk > 0 ? 1u : 0u);
-              }
-            // the BCE of this group rewrites the dY tile of group nf - 2, whose
-            // store may be the latest one issued: every store must have read its
-            // tile before the BCE is released (the forward's MMAs run meanwhile)
-            bulk_wait_read<0>();
+#pragma unroll
+            for (int kk = 0; kk < kK / 16; ++kk) {
+              const uint64_t ad =
+                  make_sdesc(WG(s) + (uint32_t)((kk / 4) * MW * 128 + (kk % 4) * 32), 16, 1024, kLayoutSw128);
+              const uint64_t bd = make_sdesc(XG(s) + (uint32_t)(kk * 16 * 128), (uint32_t)kK * 128, 1024, kLayoutSw128);
+              mma_ws(F(s), ad, bd, idesc_f, kk > 0 ? 1u : 0u);
+            }
             mma_commit(&fwd_full[s]);
           }
           __syncwarp();
@@ -243,30 +266,22 @@ __global__ void __launch_bounds__(kStepThreads, 1)
       if (nd < nf) {
         const int s = nd & 1;
         const bool rdy = __shfl_sync(0xffffffffu,
-                                     lane == 0 ? (mbar_try_wait(&dy_full[s], (nd >> 1) & 1) &&
-                                                  mbar_try_wait(&tmem_empty[s], ((nd >> 1) & 1) ^ 1))
+                                     lane == 0 ? (mbar_test_wait(&dy_full[s], (nd >> 1) & 1) &&
+                                                  mbar_test_wait(&tmem_empty[s], ((nd >> 1) & 1) ^ 1))
                                                : false,
                                      0);
         if (rdy) {
           if (lane == 0) {
             tc_fence_after();
             for (int kk = 0; kk < Bp / 16; ++kk) {
-              const int b = kk * 16;
-              const uint64_t ad =
-                  make_sdesc(XG(s) + (uint32_t)((b / 64) * kK * 128 + (kk % 4) * 32), 16, 1024, kLayoutSw128);
-              const uint64_t bd = make_sdesc(base + DY(s) + (uint32_t)(b * RB), 16, 8 * RB, layout_for_rows(RB));
-              mma_ss<false>(D(s), ad, bd, idesc_w, kk > 0 ? 1u : 0u);
+              const uint64_t ad = make_sdesc(base + DY(s) + (uint32_t)((kk / 4) * MW * 128 + (kk % 4) * 32), 16, 1024,
+                                             kLayoutSw128);
+              const uint64_t bd =
+                  make_sdesc(XG(s) + (uint32_t)((kk / 4) * kK * 128 + (kk % 4) * 32), 16, 1024, kLayoutSw128);
+              mma_ws(D(s), ad, bd, idesc_w, kk > 0 ? 1u : 0u);
             }
             mma_commit(&dw_full[s]);
             mma_commit(&empty[s]);
-            // the group's gradient tile to the dX pass's buffer: columns of its
-            // item (64 / G consecutive groups, 64 labels), the item's Bp rows
-            {
-              const int64_t g = gb + nd;
-              constexpr int NG = 64 / kG;
-              tma_store_2d(&tm_dy, base + DY(s), (int)(g % NG) * kG, (int)((g / NG) * Bp));
-            }
-            bulk_commit();
           }
           __syncwarp();
           ++nd;
@@ -288,107 +303,150 @@ __global__ void __launch_bounds__(kStepThreads, 1)
       }
     }
     // Also after an abort: the CTA frees TMEM and exits only once every MMA it
-    // issued has finished writing TMEM and reading shared memory, and its stores
-    // are complete.
-    if (lane == 0) {
-      mma_commit(done);
-      bulk_wait_all();
-    }
+    // issued has finished writing TMEM and reading shared memory.
+    if (lane == 0) mma_commit(done);
     __syncwarp();
     (void)__all_sync(0xffffffffu, mbar_wait(done, 0));
   } else {
     // ------------------------------------------------------------- epilogue
-    // warp (q, hh): TMEM lane quarter q, label columns [hh*CH, hh*CH + CH)
+    // warp (q, hh): TMEM lane quarter q, half hh of the quarter's columns
     const int ew = w - kStepMma - 1, q = w & 3, hh = ew >> 2;
-    const int r = q * 32 + lane;  // row inside a 128-row tile (and dW slot)
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-    const float scale = a.grad_scale;
+    // this thread's label m (a row of the MW-row products), its run of nct batch
+    // rows from b0 (logits) and of NSL slots from s0 (dW)
+    const int m = MW == 32 ? lane : (q & 1) * 32 + lane;
+    const bool mvalid = m < kG;
+    const int nct = (int)f_cols / 2;
+    const int b0 = (MW == 32 ? q * (Bp / 4) : (q >> 1) * (Bp / 2)) + hh * nct;
+    constexpr int NSL = (int)d_cols / 2;
+    constexpr int NCT_MAX = MW == 32 ? 32 : 64;
+    const int s0 = (MW == 32 ? q * (kK / 4) : (q >> 1) * (kK / 2)) + hh * NSL;
+    const float scale = a.grad_scale, hs = 0.5f * scale;
+    const int live = min(nct, sh.B - b0);  // rows of the run below B (may be <= 0)
     float loss_acc = 0.f;
-    // this thread's positives (tail-local ids), one batch row per 128-row tile
-    int pos[2][kMaxPosReg];
-    int npos[2] = {0, 0}, pbeg[2] = {0, 0};
-#pragma unroll
-    for (int t = 0; t < 2; ++t) {
-      const int b = t * 128 + r;
-      if (t < n_bt && b < sh.B) {
-        pbeg[t] = a.pos_ptr[b];
-        npos[t] = a.pos_ptr[b + 1] - pbeg[t];
+    // cursor of batch row rb over its positives (ids ascending): the first one at or
+    // after the current group's first label
+    const int rb = ew * 32 + lane;
+    int cur = 0, cend = 0, nid = INT_MAX;
+    if (rb < sh.B) {
+      cur = a.pos_ptr[rb];
+      cend = a.pos_ptr[rb + 1];
+      const int first = (int)(gb * kG);
+      int lo = cur, hi = cend;
+      while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (a.pos_ids[mid] < first) lo = mid + 1;
+        else hi = mid;
       }
-#pragma unroll
-      for (int e = 0; e < kMaxPosReg; ++e) pos[t][e] = e < npos[t] ? a.pos_ids[pbeg[t] + e] : -1;
+      cur = lo;
+      nid = cur < cend ? a.pos_ids[cur] : INT_MAX;
     }
-    auto bce = [&](int i) -> bool {
-      const int64_t g = gb + i;
-      const int s = i & 1;
-      if (!wait_or_abort(&fwd_full[s], (i >> 1) & 1, abort_flag)) return false;
-      tc_fence_after();
-      const int64_t l0 = g * kG + hh * CH;  // first label of this warp's columns
-      uint8_t* dyrow = gbase + DY(s);
-      // every logit of this thread's columns in both batch tiles is requested from
-      // TMEM before the first is used: one load latency per group, not one per chunk
-      constexpr int NC = CH < 16 ? CH : 16;
-      float zall[2][CH];
-#pragma unroll
-      for (int t = 0; t < 2; ++t) {
-        if (t < n_bt) {
-#pragma unroll
-          for (int c = 0; c < CH; c += 16) {
-            if constexpr (NC == 8) tmem_ld8(F(s) + lane_off + (uint32_t)(t * kG + hh * CH + c), &zall[t][c]);
-            else tmem_ld16(F(s) + lane_off + (uint32_t)(t * kG + hh * CH + c), *reinterpret_cast<float(*)[16]>(&zall[t][c]));
-          }
-        }
+    // Bit masks of group i's positives into the W_g space of its stage (free once
+    // the forward has read it): word [warp w'][label j] holds bit l for batch row
+    // 32 w' + l.  Each warp writes only its own words, whole.
+    auto build = [&](int i) {
+      const int lo = (int)((gb + i) * kG), hi = lo + kG;
+      uint64_t lm = 0;  // labels of the group that are positive in row rb
+      while (nid < hi) {
+        if (nid >= lo) lm |= 1ull << (nid - lo);
+        ++cur;
+        nid = cur < cend ? a.pos_ids[cur] : INT_MAX;
       }
+      const uint32_t any_lo = __reduce_or_sync(0xffffffffu, (uint32_t)lm);
+      const uint32_t any_hi = MW == 64 ? __reduce_or_sync(0xffffffffu, (uint32_t)(lm >> 32)) : 0u;
+      uint32_t w0 = 0, w1 = 0;
+      for (uint32_t r = any_lo; r; r &= r - 1) {
+        const int j = __ffs(r) - 1;
+        const uint32_t bj = __ballot_sync(0xffffffffu, (uint32_t)(lm >> j) & 1u);
+        if (j == lane) w0 = bj;
+      }
+      for (uint32_t r = any_hi; r; r &= r - 1) {
+        const int j = __ffs(r) - 1;
+        const uint32_t bj = __ballot_sync(0xffffffffu, (uint32_t)(lm >> (32 + j)) & 1u);
+        if (j == lane) w1 = bj;
+      }
+      if (ew * 32 < Bp) {
+        uint32_t* mk = reinterpret_cast<uint32_t*>(gbase + Lo.wg[i & 1]) + ew * MW;
+        mk[lane] = w0;
+        if constexpr (MW == 64) mk[32 + lane] = w1;
+      }
+    };
+    // group i's dY^T tile to the dX pass's buffer (epilogue thread 0, once every
+    // epilogue warp has written it): the G label rows of its item (64 / G
+    // consecutive groups, 64 labels), one box per 64 batch columns
+    const bool storer = ew == 0 && lane == 0;
+    auto store_dy = [&](int i) {
+      const int64_t g = gb + i;
+      const int row0 = (int)((g / NGI) * 64 + (g % NGI) * kG);
+      for (int blk = 0; blk < Bp / 64; ++blk)
+        tma_store_2d(&tm_dy, base + DY(i & 1) + (uint32_t)(blk * MW * 128), 64 * blk, row0);
+      bulk_commit();
+    };
+    // BCE of group i: false (the same in every epilogue thread) when the epilogue
+    // stops, after a wait ran out here or earlier.  Its barrier also orders the
+    // stores: the tile of group i - 2 (this stage) has been read before anyone
+    // writes the stage again, and group i - 1's tile is complete when it is stored.
+    auto bce = [&](int i, bool failed) -> bool {
+      const int s = i & 1;
+      bool bad = failed || !__all_sync(0xffffffffu, wait_or_abort(&fwd_full[s], (i >> 1) & 1, abort_flag));
+      if (!bad) build(i);
+      if (storer) bulk_wait_read<0>();
+      if (named_bar_or(1, kStepEpiThreads, bad || *abort_flag)) return false;
+      if (storer && i >= 1) store_dy(i - 1);
+      tc_fence_after();
+      float z[NCT_MAX];
+#pragma unroll
+      for (int c = 0; c < NCT_MAX; c += 16)
+        if (c < nct) tmem_ld16(F(s) + lane_off + (uint32_t)(hh * nct + c), *reinterpret_cast<float(*)[16]>(&z[c]));
       tmem_wait_ld();
+      const uint32_t* mk = reinterpret_cast<const uint32_t*>(gbase + Lo.wg[s]);
+      uint64_t ym = mk[(b0 >> 5) * MW + m];
+      if (nct > 32) ym |= (uint64_t)mk[((b0 >> 5) + 1) * MW + m] << 32;
+      ym >>= (b0 & 31);
+      uint8_t* dyt = gbase + DY(s);
 #pragma unroll
-      for (int t = 0; t < 2; ++t) {
-        if (t >= n_bt) break;
-        const int b = t * 128 + r;
-        const bool live = b < sh.B;
-        const float sl = live ? scale : 0.f, hs = 0.5f * sl;  // rows beyond B get dY = 0
-        uint32_t ym = 0;
+      for (int c = 0; c < NCT_MAX; c += 16) {
+        if (c >= nct) break;
+        // y = 0 everywhere first (positives are rare), then the few positive
+        // rows are corrected: dY -= scale, loss -= z
+        float dyv[16], relu = 0.f, prod = 1.f, zy = 0.f;
+        if (c + 16 <= live) {
 #pragma unroll
-        for (int e = 0; e < kMaxPosReg; ++e) {
-          const int64_t l = (int64_t)pos[t][e] - l0;
-          if (pos[t][e] >= 0 && l >= 0 && l < CH) ym |= 1u << l;
+          for (int e = 0; e < 16; ++e) {
+            const float th = tanh_approx(0.5f * z[c + e]);  // sigma(z) = (1 + th) / 2
+            dyv[e] = fmaf(hs, th, hs);                      // scale * sigma(z)
+            relu += fmaxf(z[c + e], 0.f);
+            prod *= fmaf(0.5f, fabsf(th), 0.5f);            // sigma(|z|)
+          }
+        } else {  // the run reaches past B: those rows get dY = 0 and no loss
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const bool lv = c + e < live;
+            const float th = tanh_approx(0.5f * z[c + e]);
+            dyv[e] = lv ? fmaf(hs, th, hs) : 0.f;
+            relu += lv ? fmaxf(z[c + e], 0.f) : 0.f;
+            prod *= lv ? fmaf(0.5f, fabsf(th), 0.5f) : 1.f;
+          }
         }
-        for (int e = kMaxPosReg; e < npos[t]; ++e) {  // rows with many positives
-          const int64_t l = (int64_t)a.pos_ids[pbeg[t] + e] - l0;
-          if (l >= 0 && l < CH) ym |= 1u << l;
+        const uint32_t yc = (uint32_t)(ym >> c) & 0xFFFFu;
+        if (yc) {
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            if ((yc >> e) & 1u) {
+              dyv[e] -= scale;
+              zy += z[c + e];
+            }
         }
+        // softplus(z) - z y = max(z, 0) - log sigma(|z|) - z y
+        if (mvalid) loss_acc += relu - zy - __logf(prod);
+        const int b = b0 + c;
+        const uint32_t row = (uint32_t)((b >> 6) * MW * 128 + m * 128);
 #pragma unroll
-        for (int c = 0; c < CH; c += 16) {
-          const float* z = &zall[t][c];
-          // y = 0 everywhere first (positives are rare), then the few positive
-          // columns are corrected: dY -= scale, loss -= z.
-          float dyv[16], relu = 0.f, prod = 1.f;
-#pragma unroll
-          for (int e = 0; e < NC; ++e) {
-            const float th = tanh_approx(0.5f * z[e]);   // sigma(z) = (1 + th) / 2
-            dyv[e] = fmaf(hs, th, hs);                   // scale * sigma(z)
-            relu += fmaxf(z[e], 0.f);
-            prod *= fmaf(0.5f, fabsf(th), 0.5f);         // sigma(|z|)
-          }
-          float zy = 0.f;
-          const uint32_t yc = (ym >> c) & ((1u << NC) - 1u);
-          if (yc) {
-#pragma unroll
-            for (int e = 0; e < NC; ++e)
-              if ((yc >> e) & 1u) {
-                dyv[e] -= sl;
-                zy += z[e];
-              }
-          }
-          // softplus(z) - z y = max(z, 0) - log sigma(|z|) - z y
-          if (live) loss_acc += relu - zy - __logf(prod);
-#pragma unroll
-          for (int hq = 0; hq < NC / 8; ++hq) {
-            const uint4 v = make_uint4(pack_bf16x2(dyv[8 * hq], dyv[8 * hq + 1]),
-                                       pack_bf16x2(dyv[8 * hq + 2], dyv[8 * hq + 3]),
-                                       pack_bf16x2(dyv[8 * hq + 4], dyv[8 * hq + 5]),
-                                       pack_bf16x2(dyv[8 * hq + 6], dyv[8 * hq + 7]));
-            const int col = hh * CH + c + 8 * hq;
-            *reinterpret_cast<uint4*>(dyrow + swz_rows((uint32_t)(b * RB + col * 2), RB)) = v;  // rows past B: zeros
-          }
+        for (int hq = 0; hq < 2; ++hq) {
+          const uint4 v = make_uint4(pack_bf16x2(dyv[8 * hq], dyv[8 * hq + 1]), pack_bf16x2(dyv[8 * hq + 2], dyv[8 * hq + 3]),
+                                     pack_bf16x2(dyv[8 * hq + 4], dyv[8 * hq + 5]),
+                                     pack_bf16x2(dyv[8 * hq + 6], dyv[8 * hq + 7]));
+          *reinterpret_cast<uint4*>(dyt + sw128(row + (uint32_t)((((b & 63) >> 3) + hq) * 16))) = v;
         }
       }
       fence_proxy_async_smem();
@@ -397,61 +455,58 @@ __global__ void __launch_bounds__(kStepThreads, 1)
       if (lane == 0) mbar_arrive(&dy_full[s]);
       return true;
     };
+    // dW readout of group i: this thread's label row, NSL consecutive slots, as
+    // 16-byte vectors.  False (the same in the whole warp) when a wait ran out.
     auto readout = [&](int i) -> bool {
-      const int64_t g = gb + i;
       const int s = i & 1;
-      // the update's first W and momentum values do not depend on dW: their loads
-      // are in flight while the dW product finishes
-      constexpr int NC0 = CH < 16 ? CH : 16;
-      float wv0[NC0], mv0[NC0];
+      const int64_t o = ((gb + i) * kG + m) * kK + s0;  // dW[label][slot s0]
+      // the update's W and momentum values do not depend on dW: their loads are in
+      // flight while the dW product finishes
+      uint4 wv[NSL / 8], mv[NSL / 8];
       if constexpr (kUpd > 0) {
-        if (r < kK) {
-          const int64_t o = (g * kG + hh * CH) * kK + r;
+        if (mvalid) {
 #pragma unroll
-          for (int e = 0; e < NC0; ++e) {
-            wv0[e] = __bfloat162float(W[o + (int64_t)e * kK]);
-            mv0[e] = kUpd == 2 ? __bfloat162float(a.M[o + (int64_t)e * kK]) : 0.f;
+          for (int c = 0; c < NSL / 8; ++c) {
+            wv[c] = *reinterpret_cast<const uint4*>(W + o + 8 * c);
+            mv[c] = kUpd == 2 ? *reinterpret_cast<const uint4*>(a.M + o + 8 * c) : make_uint4(0, 0, 0, 0);
           }
         }
       }
-      if (!wait_or_abort(&dw_full[s], (i >> 1) & 1, abort_flag)) return false;
+      if (!__all_sync(0xffffffffu, wait_or_abort(&dw_full[s], (i >> 1) & 1, abort_flag))) return false;
       tc_fence_after();
-      // dW readout: row = slot r, columns = this warp's labels (all requested before the wait)
-      constexpr int NCR = CH < 16 ? CH : 16;
-      float vall[CH];
+      float v[NSL];
 #pragma unroll
-      for (int c = 0; c < CH; c += 16) {
-        if constexpr (NCR == 8) tmem_ld8(D(s) + lane_off + (uint32_t)(hh * CH + c), &vall[c]);
-        else tmem_ld16(D(s) + lane_off + (uint32_t)(hh * CH + c), *reinterpret_cast<float(*)[16]>(&vall[c]));
+      for (int c = 0; c < NSL; c += 16) {
+        if constexpr (NSL == 8) tmem_ld8(D(s) + lane_off + (uint32_t)(hh * NSL), v);
+        else tmem_ld16(D(s) + lane_off + (uint32_t)(hh * NSL + c), *reinterpret_cast<float(*)[16]>(&v[c]));
       }
       tmem_wait_ld();
+      if (mvalid) {
 #pragma unroll
-      for (int c = 0; c < CH; c += 16) {
-        constexpr int NC = NCR;
-        const float* v = &vall[c];
-        if (r < kK) {
-          const int64_t off0 = (g * kG + hh * CH + c) * kK + r;  // (label, slot r); lanes: consecutive slots
+        for (int c = 0; c < NSL / 8; ++c) {
+          float d8[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) d8[e] = v[8 * c + e];
           if constexpr (kUpd == 0) {
-#pragma unroll
-            for (int e = 0; e < NC; ++e) a.dW[off0 + (int64_t)e * kK] = __float2bfloat16_rn(v[e]);
+            *reinterpret_cast<uint4*>(a.dW + o + 8 * c) =
+                make_uint4(pack_bf16x2(d8[0], d8[1]), pack_bf16x2(d8[2], d8[3]), pack_bf16x2(d8[4], d8[5]),
+                           pack_bf16x2(d8[6], d8[7]));
           } else {
-            float wv[16], mv[16];
+            const __nv_bfloat16* wb = reinterpret_cast<const __nv_bfloat16*>(&wv[c]);
+            const __nv_bfloat16* mb = reinterpret_cast<const __nv_bfloat16*>(&mv[c]);
+            float mo[8], wo[8];
 #pragma unroll
-            for (int e = 0; e < NC; ++e) {
-              if (c == 0) {
-                wv[e] = wv0[e];
-                mv[e] = mv0[e];
-              } else {
-                wv[e] = __bfloat162float(W[off0 + (int64_t)e * kK]);
-                mv[e] = kUpd == 2 ? __bfloat162float(a.M[off0 + (int64_t)e * kK]) : 0.f;
-              }
+            for (int e = 0; e < 8; ++e) {
+              mo[e] = kUpd == 2 ? fmaf(a.momentum, __bfloat162float(mb[e]), d8[e]) : d8[e];
+              wo[e] = fmaf(-a.lr, mo[e], __bfloat162float(wb[e]));
             }
-#pragma unroll
-            for (int e = 0; e < NC; ++e) {
-              const float m = kUpd == 2 ? fmaf(a.momentum, mv[e], v[e]) : v[e];
-              if constexpr (kUpd == 2) a.M[off0 + (int64_t)e * kK] = __float2bfloat16_rn(m);
-              a.W_out[off0 + (int64_t)e * kK] = __float2bfloat16_rn(fmaf(-a.lr, m, wv[e]));
-            }
+            if constexpr (kUpd == 2)
+              *reinterpret_cast<uint4*>(a.M + o + 8 * c) =
+                  make_uint4(pack_bf16x2(mo[0], mo[1]), pack_bf16x2(mo[2], mo[3]), pack_bf16x2(mo[4], mo[5]),
+                             pack_bf16x2(mo[6], mo[7]));
+            *reinterpret_cast<uint4*>(a.W_out + o + 8 * c) =
+                make_uint4(pack_bf16x2(wo[0], wo[1]), pack_bf16x2(wo[2], wo[3]), pack_bf16x2(wo[4], wo[5]),
+                           pack_bf16x2(wo[6], wo[7]));
           }
         }
       }
@@ -460,21 +515,29 @@ __global__ void __launch_bounds__(kStepThreads, 1)
       if (lane == 0) mbar_arrive(&tmem_empty[s]);
       return true;
     };
-    bool ok = n_items > 0 ? bce(0) : true;
-    for (int i = 0; ok && i < n_items; ++i) {
-      if (i + 1 < n_items && !bce(i + 1)) break;
-      if (!readout(i)) break;
+    // iteration i: the BCE of group i, then the dW readout of group i - 1.  Every
+    // epilogue thread passes the same named barriers: a readout that fails stops
+    // the loop only at the next BCE's barrier.
+    bool failed = false, all_bce = true;
+    for (int i = 0; i <= n_items; ++i) {
+      if (i < n_items && !bce(i, failed)) {
+        all_bce = false;
+        break;
+      }
+      if (i >= 1 && !failed) failed = !readout(i - 1);
     }
     // deterministic loss reduction over the epilogue warps (named barrier 1)
     float v = loss_acc;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     if (lane == 0) red[ew] = v;
-    named_bar(1, 32 * kStepEpi);
-    if (ew == 0 && lane == 0) {
+    named_bar(1, kStepEpiThreads);
+    if (storer) {
       float t = 0.f;
       for (int j = 0; j < kStepEpi; ++j) t += red[j];
       a.loss_part[blockIdx.x] = t;
+      if (all_bce && n_items > 0) store_dy(n_items - 1);  // every warp has written it (barrier above)
+      bulk_wait_all();  // the CTA exits only once its stores are complete
     }
   }
   tc_fence_before();
@@ -503,11 +566,11 @@ cudaError_t launch_step_t(const v2::StepArgs& a, int grid, const void* Xt, const
   auto kern = v2::k_step2<kG, kK, kUpd>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  // the gradient buffer [n_items * Bp][64] as the stores' tensor: group g's box
-  // (G labels x Bp rows) at columns (g % NG) * G of item g / NG's rows, NG = 64 / G
+  // the gradient buffer [n_items * 64][Bp] (label rows, items of 64 / G groups) as
+  // the stores' tensor: group g's G label rows, one box per 64 batch columns
   CUtensorMap tm_dy;
   const uint64_t n_items = (uint64_t)(a.sh.n_groups + 64 / kG - 1) / (64 / kG);
-  e = tmap_2d(&tm_dy, a.dY_out, 64, n_items * a.sh.Bp, 128, kG, (uint32_t)a.sh.Bp);
+  e = tmap_2d(&tm_dy, a.dY_out, (uint64_t)a.sh.Bp, n_items * 64, (uint64_t)a.sh.Bp * 2, 64, kG);
   if (e != cudaSuccess) return e;
   kern<<<grid, v2::kStepThreads, smem, st>>>(a, static_cast<const __nv_bfloat16*>(Xt),
                                              static_cast<const __nv_bfloat16*>(W), tm_dy);
