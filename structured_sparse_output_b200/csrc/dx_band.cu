@@ -209,17 +209,21 @@ __global__ void __launch_bounds__(kDxThreads, 1)
       tc_fence_after();
       if (lane == 0) {
         const int nk = cnt(i) * (kG / 16);  // K steps of the item's present labels
+        // the fused step's tile is label rows (batch contiguous: MN-major, 64-row
+        // blocks 8 KB apart), a caller's is batch rows (labels contiguous: K-major);
+        // descriptors advance by start-address offsets (16-byte units), so that an
+        // MMA costs few instructions of this warp, which shares its scheduler with
+        // densify warps
+        const uint64_t ad0 = a.group_major ? make_sdesc(DYS(st), 64 * 128, 1024, kLayoutSw128)
+                                           : make_sdesc(DYS(st), 16, 1024, kLayoutSw128);
+        const uint32_t kstep = a.group_major ? 16 * 128 / 16 : 32 / 16;
+        const uint64_t bd0 = make_sdesc(WT(st), 16, 1024, kLayoutSw128);
         for (int t = 0; t < MT; ++t)
-          for (int kk = 0; kk < nk; ++kk) {
-            // the fused step's tile is label rows (batch contiguous: MN-major, 64-row
-            // blocks 8 KB apart), a caller's is batch rows (labels contiguous: K-major)
-            const uint64_t ad =
-                a.group_major
-                    ? make_sdesc(DYS(st) + (uint32_t)(t * 2 * 64 * 128 + kk * 16 * 128), 64 * 128, 1024, kLayoutSw128)
-                    : make_sdesc(DYS(st) + (uint32_t)(t * 128 * 128 + kk * 32), 16, 1024, kLayoutSw128);
-            const uint64_t bd = make_sdesc(WT(st) + (uint32_t)(kk * 32), 16, 1024, kLayoutSw128);
-            mma_ss<false>(tmem + (uint32_t)(t * 256), ad, bd, idesc, (i > 0 || kk > 0) ? 1u : 0u);
-          }
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            if (kk < nk)
+              mma_ss<false>(tmem + (uint32_t)(t * 256), ad0 + (uint64_t)(t * 1024 + kk * kstep), bd0 + (uint64_t)(kk * 2),
+                            idesc, (i > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&empty[st]);
         mma_commit(&wt_empty[st]);
       }

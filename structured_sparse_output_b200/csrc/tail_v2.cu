@@ -238,7 +238,9 @@ __global__ void __launch_bounds__(kStepThreads, 1)
     const uint32_t idesc_f = make_idesc(1, 0, 1, MW, (uint32_t)Bp);
     const uint32_t idesc_w = make_idesc(1, 0, 0, MW, kK);
     int nf = 0, nd = 0;
-    uint64_t t_last = globaltimer_ns();
+    // the timer is read only while nothing is ready (a read costs hundreds of
+    // cycles): t_idle is when the current idle stretch began, 0 after progress
+    uint64_t t_idle = 0;
     const uint64_t limit = g_wait_limit_ns;
     while (nd < n_items) {
       if (*abort_flag) break;
@@ -250,12 +252,16 @@ __global__ void __launch_bounds__(kStepThreads, 1)
           if (lane == 0) {
             tc_fence_after();
 #pragma unroll
-            for (int kk = 0; kk < kK / 16; ++kk) {
-              const uint64_t ad =
-                  make_sdesc(WG(s) + (uint32_t)((kk / 4) * MW * 128 + (kk % 4) * 32), 16, 1024, kLayoutSw128);
-              const uint64_t bd = make_sdesc(XG(s) + (uint32_t)(kk * 16 * 128), (uint32_t)kK * 128, 1024, kLayoutSw128);
-              mma_ws(F(s), ad, bd, idesc_f, kk > 0 ? 1u : 0u);
-            }
+            // descriptors advance by constant start-address offsets (16-byte units):
+            // the issuing warp shares its scheduler with busy warps, so each MMA
+            // costs only a few instructions
+            const uint64_t ad0 = make_sdesc(WG(s), 16, 1024, kLayoutSw128);
+            const uint64_t bd0 = make_sdesc(XG(s), (uint32_t)kK * 128, 1024, kLayoutSw128);
+            const uint32_t f = F(s);
+#pragma unroll
+            for (int kk = 0; kk < kK / 16; ++kk)
+              mma_ws(f, ad0 + (uint64_t)(((kk / 4) * MW * 128 + (kk % 4) * 32) >> 4), bd0 + (uint64_t)(kk * 128), idesc_f,
+                     kk > 0 ? 1u : 0u);
             mma_commit(&fwd_full[s]);
           }
           __syncwarp();
@@ -273,12 +279,19 @@ __global__ void __launch_bounds__(kStepThreads, 1)
         if (rdy) {
           if (lane == 0) {
             tc_fence_after();
-            for (int kk = 0; kk < Bp / 16; ++kk) {
-              const uint64_t ad = make_sdesc(base + DY(s) + (uint32_t)((kk / 4) * MW * 128 + (kk % 4) * 32), 16, 1024,
-                                             kLayoutSw128);
-              const uint64_t bd =
-                  make_sdesc(XG(s) + (uint32_t)((kk / 4) * kK * 128 + (kk % 4) * 32), 16, 1024, kLayoutSw128);
-              mma_ws(D(s), ad, bd, idesc_w, kk > 0 ? 1u : 0u);
+            const uint64_t ad0 = make_sdesc(base + DY(s), 16, 1024, kLayoutSw128);
+            const uint64_t bd0 = make_sdesc(XG(s), 16, 1024, kLayoutSw128);
+            const uint32_t d = D(s);
+            auto dw_mma = [&](int kk) {
+              mma_ws(d, ad0 + (uint64_t)(((kk / 4) * MW * 128 + (kk % 4) * 32) >> 4),
+                     bd0 + (uint64_t)(((kk / 4) * kK * 128 + (kk % 4) * 32) >> 4), idesc_w, kk > 0 ? 1u : 0u);
+            };
+            if (Bp == 256) {
+#pragma unroll
+              for (int kk = 0; kk < 16; ++kk) dw_mma(kk);
+            } else {
+#pragma unroll
+              for (int kk = 0; kk < 8; ++kk) dw_mma(kk);
             }
             mma_commit(&dw_full[s]);
             mma_commit(&empty[s]);
@@ -289,9 +302,11 @@ __global__ void __launch_bounds__(kStepThreads, 1)
         }
       }
       if (did) {
-        t_last = globaltimer_ns();
+        t_idle = 0;
       } else {
-        if (globaltimer_ns() - t_last > limit) {
+        const uint64_t now = globaltimer_ns();
+        if (t_idle == 0) t_idle = now;
+        if (now - t_idle > limit) {
           if (lane == 0) {
             *abort_flag = 1;
             record_error(kErrTimeout);
