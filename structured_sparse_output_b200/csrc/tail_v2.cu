@@ -8,12 +8,12 @@
 // or every slot (dW: N = k):
 //   forward  logits_g^T [MW, Bp] = W_g [MW, k] . Xg^T     (K = k)
 //   dW       dW_g^T     [MW, k]  = dY_g^T [MW, Bp] . Xg   (K = Bp)
-//   warps 0-3  producers: the gather-once tile Xg = X[:, I_g] (k rows of X^T) and
-//              the G x k weight block, staged with cp.async into a 2-stage ring
-//              (all four warps fill the stage of each group);
-//   warp 4     MMA issuer (one thread): issues each group's forward and dW
+//   warp 0     MMA issuer (one thread): issues each group's forward and dW
 //              product as soon as its inputs are ready;
-//   warps 5-12 epilogue: each thread owns one label and a run of batch rows of the
+//   warps 1-3  producers: the gather-once tile Xg = X[:, I_g] (k rows of X^T) and
+//              the G x k weight block, staged with cp.async into a 2-stage ring
+//              (the three warps fill the stage of each group);
+//   warps 4-11 epilogue: each thread owns one label and a run of batch rows of the
 //              logits; they leave TMEM only as the BCE gradient dY^T (bf16, into
 //              shared memory: the dW operand, and the tile that epilogue thread 0
 //              writes to the gradient buffer of the dX pass with TMA stores).  The
@@ -103,10 +103,15 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
 }
 
 // ============================================================ k_step2
-constexpr int kStepProd = 4;       // producer warps: two per ring stage
-constexpr int kStepMma = kStepProd;  // warp id of the MMA issuer
+// Warp roles.  The MMA issuer (warp 0) shares its scheduler only with two
+// epilogue warps: the producers' stream of cp.async fills the memory-instruction
+// queue of theirs, and each barrier test of the issuer would wait behind it.
+constexpr int kStepMma = 0;        // warp id of the MMA issuer
+constexpr int kStepProd0 = 1;      // producer warps 1-3
+constexpr int kStepProd = 3;
+constexpr int kStepEpi0 = 4;       // epilogue warps 4-11
 constexpr int kStepEpi = 8;        // epilogue warps: 4 lane quarters x 2 column halves
-constexpr int kStepThreads = 32 * (kStepProd + 1 + kStepEpi);  // producers, MMA warp, epilogue warps
+constexpr int kStepThreads = 32 * (1 + kStepProd + kStepEpi);
 constexpr int kStepEpiThreads = 32 * kStepEpi;
 
 template <int kG, int kK, int kUpd>
@@ -172,15 +177,17 @@ __global__ void __launch_bounds__(kStepThreads, 1)
   const int64_t ge = (int64_t)(blockIdx.x + 1) * sh.n_groups / gridDim.x;
   const int n_items = (int)(ge - gb);
 
-  if (w < kStepProd) {
+  if (w >= kStepProd0 && w < kStepProd0 + kStepProd) {
     // ------------------------------------------------- cp.async producers
-    // all four warps fill the stage of every item i (stage i & 1); warp part
-    // copies every fourth group of four rows.  Lane (rg, sub) copies the 16-byte
-    // chunk sub of every 128-byte segment of its rows, so that 8 consecutive lanes
-    // read one segment; the feature indices of its rows sit in registers.
+    // the three warps fill the stage of every item i (stage i & 1); warp part
+    // copies the groups of four rows part, part + 3, ...  Lane (rg, sub) copies
+    // the 16-byte chunk sub of every 128-byte segment of its rows, so that 8
+    // consecutive lanes read one segment; the feature indices of its rows sit in
+    // registers.
     constexpr int P = kStepProd;
-    constexpr int kRows = kRowsPerThr / P;
-    const int part = w, ht = lane;
+    constexpr int kQuads = kK / 4;                 // groups of four rows
+    constexpr int kRows = (kQuads + P - 1) / P;    // per warp (the last may be short)
+    const int part = w - kStepProd0, ht = lane;
     const int sub = ht & 7, rg = ht >> 3;
     for (int i = 0; i < n_items; ++i) {
       const int64_t g = gb + i;
@@ -196,11 +203,13 @@ __global__ void __launch_bounds__(kStepThreads, 1)
       // the index loads are in flight while this half waits for its stage
       int idx_cur[kRows];
 #pragma unroll
-      for (int m = 0; m < kRows; ++m) idx_cur[m] = a.idx[g * kK + rg + 4 * (m * P + part)];
+      for (int m = 0; m < kRows; ++m)
+        idx_cur[m] = m * P + part < kQuads ? a.idx[g * kK + rg + 4 * (m * P + part)] : 0;
       if (!wait_or_abort(&empty[half], ((i >> 1) & 1) ^ 1, abort_flag)) break;
       const int nbb = Bp / 64;
 #pragma unroll
       for (int m = 0; m < kRows; ++m) {
+        if (m * P + part >= kQuads) break;
         const int sl = rg + 4 * (m * P + part);
         const __nv_bfloat16* src = Xt + (int64_t)idx_cur[m] * Bp + sub * 8;
         const uint32_t dst = xg + sw128((uint32_t)(sl * 128 + sub * 16));  // swizzle is the same in every block
@@ -243,7 +252,6 @@ __global__ void __launch_bounds__(kStepThreads, 1)
     uint64_t t_idle = 0;
     const uint64_t limit = g_wait_limit_ns;
     while (nd < n_items) {
-      if (*abort_flag) break;
       bool did = false;
       if (nf < n_items && nf <= nd + 1) {
         const int s = nf & 1;
@@ -251,7 +259,6 @@ __global__ void __launch_bounds__(kStepThreads, 1)
         if (rdy) {
           if (lane == 0) {
             tc_fence_after();
-#pragma unroll
             // descriptors advance by constant start-address offsets (16-byte units):
             // the issuing warp shares its scheduler with busy warps, so each MMA
             // costs only a few instructions
@@ -304,6 +311,7 @@ __global__ void __launch_bounds__(kStepThreads, 1)
       if (did) {
         t_idle = 0;
       } else {
+        if (*abort_flag) break;
         const uint64_t now = globaltimer_ns();
         if (t_idle == 0) t_idle = now;
         if (now - t_idle > limit) {
@@ -314,7 +322,8 @@ __global__ void __launch_bounds__(kStepThreads, 1)
           __syncwarp();
           break;
         }
-        __nanosleep(32);
+        // no sleep here: a suspended issuer wakes far later than the barriers
+        // complete, and the tensor core would wait for it
       }
     }
     // Also after an abort: the CTA frees TMEM and exits only once every MMA it
@@ -325,7 +334,7 @@ __global__ void __launch_bounds__(kStepThreads, 1)
   } else {
     // ------------------------------------------------------------- epilogue
     // warp (q, hh): TMEM lane quarter q, half hh of the quarter's columns
-    const int ew = w - kStepMma - 1, q = w & 3, hh = ew >> 2;
+    const int ew = w - kStepEpi0, q = w & 3, hh = ew >> 2;
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     // this thread's label m (a row of the MW-row products), its run of nct batch
     // rows from b0 (logits) and of NSL slots from s0 (dW)
