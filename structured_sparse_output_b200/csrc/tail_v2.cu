@@ -121,7 +121,6 @@ __global__ void __launch_bounds__(kStepThreads, 1)
   extern __shared__ __align__(1024) uint8_t smem[];
   constexpr int MW = step_mw(kG);     // rows of the weight-stationary MMAs
   constexpr int NGI = 64 / kG;        // groups per 64-label item of the gradient buffer
-  constexpr int kRowsPerThr = kK / 4;
   const TailShape sh = a.sh;
   const int Bp = sh.Bp;
   const StepLayout Lo = step_layout(Bp, kK, kG);

@@ -125,6 +125,8 @@ STEP_CASES = [
     dict(B=100, d=256, n_groups=120, G=16, k=64, dtype="bf16", H=0, p=5),   # one batch tile, G = 16
     dict(B=1, d=256, n_groups=40, G=32, k=64, dtype="bf16", H=16, p=3),     # a batch of one row
     dict(B=37, d=256, n_groups=1, G=32, k=64, dtype="bf16", H=0, p=2),      # a single group
+    dict(B=200, d=384, n_groups=301, G=16, k=128, dtype="bf16", H=0, p=6),  # CTA pairs, G = 16
+    dict(B=256, d=512, n_groups=5, G=32, k=128, dtype="bf16", H=0, p=4),    # fewer groups than CTA pairs
 ]
 
 
@@ -290,6 +292,7 @@ SGD_CASES = [
     dict(B=256, d=768, n_groups=300, G=64, k=128, dtype="bf16", H=0, p=8, lr=8.0, mu=0.9),
     dict(B=130, d=384, n_groups=250, G=32, k=64, dtype="bf16", H=0, p=5, lr=16.0, mu=0.0),
     dict(B=100, d=256, n_groups=120, G=16, k=64, dtype="bf16", H=0, p=5, lr=12.0, mu=0.5),
+    dict(B=180, d=384, n_groups=211, G=16, k=128, dtype="bf16", H=0, p=5, lr=10.0, mu=0.9),
 ]
 
 
