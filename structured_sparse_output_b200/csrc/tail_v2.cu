@@ -54,10 +54,11 @@ __host__ __device__ constexpr int step_mw(int G) { return G <= 32 ? 32 : 64; }
 // ------------------------------------------------------------ smem layouts
 // Per stage: Xg [Bp/64][k][64] (slot rows, 64 batch columns per 128-byte row),
 // W_g [k/64][MW][64] (label rows, 64 slots per row) and dY^T [Bp/64][MW][64]
-// (label rows, 64 batch columns per row), all 128B-swizzled.  After the forward
-// has read W_g, its space holds the group's positive-label bit masks.
+// (label rows, 64 batch columns per row), all 128B-swizzled, and the group's
+// positive-label bit masks [Bp/32][MW]: their own space for MW = 32, for MW = 64
+// (no room left) the W_g space once the forward has read it.
 struct StepLayout {
-  uint32_t xg[2], wg[2], dy[2], bars, total;
+  uint32_t xg[2], wg[2], dy[2], mk[2], bars, total;
 };
 __host__ __device__ inline StepLayout step_layout(int Bp, int k, int G) {
   StepLayout L;
@@ -69,6 +70,14 @@ __host__ __device__ inline StepLayout step_layout(int Bp, int k, int G) {
   for (int s = 0; s < 2; ++s) { L.xg[s] = off; off += xg; }
   for (int s = 0; s < 2; ++s) { L.wg[s] = off; off += wg; }
   for (int s = 0; s < 2; ++s) { L.dy[s] = off; off += dy; }
+  for (int s = 0; s < 2; ++s) {
+    if (MW == 32) {
+      L.mk[s] = off;
+      off += (uint32_t)((Bp / 32) * MW * 4);
+    } else {
+      L.mk[s] = L.wg[s];
+    }
+  }
   L.bars = off;
   off += 256;
   L.total = off + 1024;
@@ -389,7 +398,7 @@ __global__ void __launch_bounds__(kStepThreads, 1)
         if (j == lane) w1 = bj;
       }
       if (ew * 32 < Bp) {
-        uint32_t* mk = reinterpret_cast<uint32_t*>(gbase + Lo.wg[i & 1]) + ew * MW;
+        uint32_t* mk = reinterpret_cast<uint32_t*>(gbase + Lo.mk[i & 1]) + ew * MW;
         mk[lane] = w0;
         if constexpr (MW == 64) mk[32 + lane] = w1;
       }
@@ -406,23 +415,35 @@ __global__ void __launch_bounds__(kStepThreads, 1)
       bulk_commit();
     };
     // BCE of group i: false (the same in every epilogue thread) when the epilogue
-    // stops, after a wait ran out here or earlier.  Its barrier also orders the
-    // stores: the tile of group i - 2 (this stage) has been read before anyone
-    // writes the stage again, and group i - 1's tile is complete when it is stored.
-    auto bce = [&](int i, bool failed) -> bool {
+    // stops, after a wait ran out earlier.  Its barrier also orders the stores: the
+    // tile of group i - 2 (this stage) has been read before anyone writes the stage
+    // again, and group i - 1's tile is complete when it is stored.
+    auto bce = [&](int i, bool& failed) -> bool {
       const int s = i & 1;
-      bool bad = failed || !__all_sync(0xffffffffu, wait_or_abort(&fwd_full[s], (i >> 1) & 1, abort_flag));
-      if (!bad) build(i);
+      // With their own mask space (MW = 32), the masks, the barrier and the
+      // previous group's stores do not depend on the forward and run while it does;
+      // for MW = 64 the masks take the W_g space after the forward.  A wait that runs
+      // out stops the loop at the next barrier (every warp passes the same barriers).
+      if constexpr (MW == 64) {
+        if (!failed && !__all_sync(0xffffffffu, wait_or_abort(&fwd_full[s], (i >> 1) & 1, abort_flag))) failed = true;
+      }
+      if (!failed) build(i);
       if (storer) bulk_wait_read<0>();
-      if (named_bar_or(1, kStepEpiThreads, bad || *abort_flag)) return false;
+      if (named_bar_or(1, kStepEpiThreads, failed || *abort_flag)) return false;
       if (storer && i >= 1) store_dy(i - 1);
+      if constexpr (MW == 32) {
+        if (!__all_sync(0xffffffffu, wait_or_abort(&fwd_full[s], (i >> 1) & 1, abort_flag))) {
+          failed = true;
+          return true;
+        }
+      }
       tc_fence_after();
       float z[NCT_MAX];
 #pragma unroll
       for (int c = 0; c < NCT_MAX; c += 16)
         if (c < nct) tmem_ld16(F(s) + lane_off + (uint32_t)(hh * nct + c), *reinterpret_cast<float(*)[16]>(&z[c]));
       tmem_wait_ld();
-      const uint32_t* mk = reinterpret_cast<const uint32_t*>(gbase + Lo.wg[s]);
+      const uint32_t* mk = reinterpret_cast<const uint32_t*>(gbase + Lo.mk[s]);
       uint64_t ym = mk[(b0 >> 5) * MW + m];
       if (nct > 32) ym |= (uint64_t)mk[((b0 >> 5) + 1) * MW + m] << 32;
       ym >>= (b0 & 31);
