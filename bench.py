@@ -86,8 +86,10 @@ def algorithmic(wl):
 # kernel from one ncu capture (summaries under profiles/), valid only for the
 # source file it was taken on: (config, timed region) -> (bytes, source digest).
 TRAFFIC = {
-    ("670k", "tail_step"): (647.6e6, "c8e981bb0d4fe169"),
-    ("670k", "tail_dx"): (529.9e6, "697f773de5956a06"),
+    ("670k", "tail_step"): (644.4e6, "307261f4ece010ee"),
+    ("670k", "tail_dx"): (530.1e6, "2115c55101e00c65"),
+    ("8.6m", "tail_step"): (8.83e9, "307261f4ece010ee"),
+    ("8.6m", "tail_dx"): (6.82e9, "2115c55101e00c65"),
 }
 # timed region -> (source file under csrc/, kernel name in the ncu summaries)
 KERNELS = {"tail_step": ("tail_v2.cu", "k_step2"), "tail_dx": ("dx_band.cu", "k_dx_band"),
