@@ -90,6 +90,7 @@ TRAFFIC = {
     ("670k", "tail_dx"): (530.1e6, "2115c55101e00c65"),
     ("8.6m", "tail_step"): (8.83e9, "307261f4ece010ee"),
     ("8.6m", "tail_dx"): (6.82e9, "2115c55101e00c65"),
+    ("670k", "topk_score"): (187.0e6, "48974329ba8749cd"),
 }
 # timed region -> (source file under csrc/, kernel name in the ncu summaries)
 KERNELS = {"tail_step": ("tail_v2.cu", "k_step2"), "tail_dx": ("dx_band.cu", "k_dx_band"),
