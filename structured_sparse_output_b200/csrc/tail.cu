@@ -466,33 +466,36 @@ __global__ void __launch_bounds__(256) k_dx_reduce(const float* __restrict__ P, 
                                                    int d, int Bp, int B, int accumulate,
                                                    const float* __restrict__ loss_part, int n_loss, float scale,
                                                    float* __restrict__ loss) {
-  __shared__ float tile[32][33];
-  const int f0 = blockIdx.x * 32, b0 = blockIdx.y * 32;
-  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  // block: 8 feature rows x 128 batch columns; warp w sums feature f0 + w, lane l
+  // the 4 batch columns 4l.. as one 16-byte load per chunk (eight loads in flight);
+  // every element adds its chunks in ascending order
+  __shared__ float tile[8][128 + 4];
+  const int f0 = blockIdx.x * 8, b0 = blockIdx.y * 128;
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
   if (loss_part && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x < 32) loss_sum(loss_part, n_loss, scale, loss);
-  // four feature rows per thread, summed side by side so that their loads are in
-  // flight together; every element still adds its chunks in ascending order
   const int64_t cs = (int64_t)d * Bp;
-  const float* p = P + (int64_t)(f0 + ty) * Bp + b0 + tx;
-  const bool k0 = f0 + ty < d, k1 = f0 + ty + 8 < d, k2 = f0 + ty + 16 < d, k3 = f0 + ty + 24 < d;
-  float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-#pragma unroll 4
-  for (int c = 0; c < C; ++c) {
-    const float* q = p + c * cs;
-    if (k0) s0 += q[0];
-    if (k1) s1 += q[8 * Bp];
-    if (k2) s2 += q[16 * Bp];
-    if (k3) s3 += q[24 * Bp];
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (f0 + w < d) {
+    const float4* p = reinterpret_cast<const float4*>(P + (int64_t)(f0 + w) * Bp + b0) + l;
+#pragma unroll 8
+    for (int c = 0; c < C; ++c) {
+      const float4 v = p[c * (cs / 4)];
+      acc.x += v.x;
+      acc.y += v.y;
+      acc.z += v.z;
+      acc.w += v.w;
+    }
   }
-  tile[ty][tx] = s0;
-  tile[ty + 8][tx] = s1;
-  tile[ty + 16][tx] = s2;
-  tile[ty + 24][tx] = s3;
+  tile[w][4 * l] = acc.x;
+  tile[w][4 * l + 1] = acc.y;
+  tile[w][4 * l + 2] = acc.z;
+  tile[w][4 * l + 3] = acc.w;
   __syncthreads();
-  for (int i = ty; i < 32; i += 8) {
-    const int bb = b0 + i, f = f0 + tx;
+  // dX rows: eight consecutive features of one batch row per group of 8 threads
+  for (int i = threadIdx.x; i < 8 * 128; i += 256) {
+    const int bb = b0 + i / 8, f = f0 + (i & 7);
     if (bb < B && f < d) {
-      const float v = tile[tx][i];
+      const float v = tile[i & 7][i / 8];
       float* q = dX + (int64_t)bb * d + f;
       *q = accumulate ? *q + v : v;
     }
@@ -740,7 +743,7 @@ cudaError_t launch_backward_dx(const TailArgs& a, bool from_step, cudaStream_t s
 cudaError_t launch_dx_reduce(const float* P, float* dX, int C, int d, int Bp, int B, int accumulate,
                              cudaStream_t st, const float* loss_part = nullptr, int n_loss = 0,
                              float scale = 0.f, float* loss = nullptr) {
-  dim3 grid((d + 31) / 32, Bp / 32);
+  dim3 grid((d + 7) / 8, Bp / 128);
   k_dx_reduce<<<grid, 256, 0, st>>>(P, dX, C, d, Bp, B, accumulate, loss_part, n_loss, scale, loss);
   return cudaGetLastError();
 }
