@@ -10,10 +10,10 @@
 //   dW       dW_g^T     [MW, k]  = dY_g^T [MW, Bp] . Xg   (K = Bp)
 //   warp 0     MMA issuer (one thread): issues each group's forward and dW
 //              product as soon as its inputs are ready;
-//   warps 1-3  producers: the gather-once tile Xg = X[:, I_g] (k rows of X^T) and
-//              the G x k weight block, staged with cp.async into a 2-stage ring
-//              (the three warps fill the stage of each group);
-//   warps 4-11 epilogue: each thread owns one label and a run of batch rows of the
+//   producers  six warps (three for G = 64): the gather-once tile Xg = X[:, I_g]
+//              (k rows of X^T) and the G x k weight block, staged with cp.async
+//              into a 2-stage ring (all of them fill the stage of each group);
+//   epilogue   eight warps: each thread owns one label and a run of batch rows of the
 //              logits; they leave TMEM only as the BCE gradient dY^T (bf16, into
 //              shared memory: the dW operand, and the tile that epilogue thread 0
 //              writes to the gradient buffer of the dX pass with TMA stores).  The
@@ -112,19 +112,36 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
 }
 
 // ============================================================ k_step2
-// Warp roles.  The MMA issuer (warp 0) shares its scheduler only with two
-// epilogue warps: the producers' stream of cp.async fills the memory-instruction
-// queue of theirs, and each barrier test of the issuer would wait behind it.
+// Warp roles (warp w runs on scheduler w % 4, which also fixes the TMEM lane
+// quarter an epilogue warp can read).  The MMA issuer (warp 0) shares its
+// scheduler with no producer: the producers' stream of cp.async fills the
+// memory-instruction queue of theirs, and each barrier test of the issuer would
+// wait behind it.
+//   G <= 32: six producer warps (1-3, 5-7, two on each of schedulers 1-3) keep
+//            more gathered rows in flight; epilogue warps 4 and 8 (quarter 0), 9
+//            and 13 (1), 10 and 14 (2), 11 and 15 (3); warp 12 idles.  512 threads.
+//   G = 64:  three producer warps (1-3) and epilogue warps 4-11, 384 threads: the
+//            64-label epilogue needs the registers of the smaller block.
 constexpr int kStepMma = 0;        // warp id of the MMA issuer
-constexpr int kStepProd0 = 1;      // producer warps 1-3
-constexpr int kStepProd = 3;
-constexpr int kStepEpi0 = 4;       // epilogue warps 4-11
 constexpr int kStepEpi = 8;        // epilogue warps: 4 lane quarters x 2 column halves
-constexpr int kStepThreads = 32 * (1 + kStepProd + kStepEpi);
 constexpr int kStepEpiThreads = 32 * kStepEpi;
+__host__ __device__ constexpr int step_prod_warps(int G) { return G == 64 ? 3 : 6; }
+__host__ __device__ constexpr int step_threads(int G) { return G == 64 ? 32 * 12 : 32 * 16; }
+// producer index of warp w (-1: not a producer)
+template <int kG>
+__device__ __forceinline__ int step_prod_part(int w) {
+  if constexpr (kG == 64) return w >= 1 && w <= 3 ? w - 1 : -1;
+  else return w >= 1 && w <= 3 ? w - 1 : w >= 5 && w <= 7 ? w - 2 : -1;
+}
+// epilogue index ew = quarter + 4 * half of warp w (-1: not an epilogue warp)
+template <int kG>
+__device__ __forceinline__ int step_epi_index(int w) {
+  if constexpr (kG == 64) return w >= 4 && w <= 11 ? w - 4 : -1;
+  else return w == 4 ? 0 : w == 8 ? 4 : w >= 9 && w != 12 ? w - 8 : -1;
+}
 
 template <int kG, int kK, int kUpd>
-__global__ void __launch_bounds__(kStepThreads, 1)
+__global__ void __launch_bounds__(step_threads(kG), 1)
     k_step2(StepArgs a, const __nv_bfloat16* __restrict__ Xt, const __nv_bfloat16* __restrict__ W,
             const __grid_constant__ CUtensorMap tm_dy) {
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -150,7 +167,7 @@ __global__ void __launch_bounds__(kStepThreads, 1)
   const int w = warp_id(), lane = lane_id();
   if (threadIdx.x == 0) {
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&full[s], 32 * kStepProd);
+      mbar_init(&full[s], 32 * step_prod_warps(kG));
       mbar_init(&empty[s], 1);
       mbar_init(&fwd_full[s], 1);
       mbar_init(&dy_full[s], kStepEpi);
@@ -185,17 +202,17 @@ __global__ void __launch_bounds__(kStepThreads, 1)
   const int64_t ge = (int64_t)(blockIdx.x + 1) * sh.n_groups / gridDim.x;
   const int n_items = (int)(ge - gb);
 
-  if (w >= kStepProd0 && w < kStepProd0 + kStepProd) {
+  if (step_prod_part<kG>(w) >= 0) {
     // ------------------------------------------------- cp.async producers
-    // the three warps fill the stage of every item i (stage i & 1); warp part
-    // copies the groups of four rows part, part + 3, ...  Lane (rg, sub) copies
+    // the producer warps fill the stage of every item i (stage i & 1); warp part
+    // copies the groups of four rows part, part + P, ...  Lane (rg, sub) copies
     // the 16-byte chunk sub of every 128-byte segment of its rows, so that 8
     // consecutive lanes read one segment; the feature indices of its rows sit in
     // registers.
-    constexpr int P = kStepProd;
+    constexpr int P = step_prod_warps(kG);
     constexpr int kQuads = kK / 4;                 // groups of four rows
     constexpr int kRows = (kQuads + P - 1) / P;    // per warp (the last may be short)
-    const int part = w - kStepProd0, ht = lane;
+    const int part = step_prod_part<kG>(w), ht = lane;
     const int sub = ht & 7, rg = ht >> 3;
     for (int i = 0; i < n_items; ++i) {
       const int64_t g = gb + i;
@@ -339,10 +356,10 @@ __global__ void __launch_bounds__(kStepThreads, 1)
     if (lane == 0) mma_commit(done);
     __syncwarp();
     (void)__all_sync(0xffffffffu, mbar_wait(done, 0));
-  } else {
+  } else if (step_epi_index<kG>(w) >= 0) {
     // ------------------------------------------------------------- epilogue
     // warp (q, hh): TMEM lane quarter q, half hh of the quarter's columns
-    const int ew = w - kStepEpi0, q = w & 3, hh = ew >> 2;
+    const int ew = step_epi_index<kG>(w), q = w & 3, hh = ew >> 2;
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     // this thread's label m (a row of the MW-row products), its run of nct batch
     // rows from b0 (logits) and of NSL slots from s0 (dW)
@@ -616,7 +633,7 @@ cudaError_t launch_step_t(const v2::StepArgs& a, int grid, const void* Xt, const
   const uint64_t n_items = (uint64_t)(a.sh.n_groups + 64 / kG - 1) / (64 / kG);
   e = tmap_2d(&tm_dy, a.dY_out, (uint64_t)a.sh.Bp, n_items * 64, (uint64_t)a.sh.Bp * 2, 64, kG);
   if (e != cudaSuccess) return e;
-  kern<<<grid, v2::kStepThreads, smem, st>>>(a, static_cast<const __nv_bfloat16*>(Xt),
+  kern<<<grid, v2::step_threads(kG), smem, st>>>(a, static_cast<const __nv_bfloat16*>(Xt),
                                              static_cast<const __nv_bfloat16*>(W), tm_dy);
   return cudaGetLastError();
 }
