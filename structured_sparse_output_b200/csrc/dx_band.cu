@@ -43,21 +43,20 @@ __host__ __device__ inline int64_t n_items_of(int64_t n_groups, int G) {
 }
 
 struct DxLayout {
-  uint32_t dy, w, wt, bars, total, dy_stride, w_stride, wt_stride;
+  uint32_t dy, wt, bars, total, dy_stride, wt_stride;
 };
-// Shared memory of the dX pass: ns stages of (dY tile [rows][64], weight rows
-// [k/64][64][64], densified weight block [band][64]; 128-byte rows, 128B
-// swizzle) and the barriers.
+// Shared memory of the dX pass: ns stages of (dY tile [rows][64], densified weight
+// block [band][64]; 128-byte rows, 128B swizzle) and the barriers.  The weight
+// rows are read by the densify warps straight from global memory (L2), so that a
+// third stage fits.
 __host__ __device__ inline DxLayout dx_layout(int rows, int band, int k, int ns) {
+  (void)k;
   DxLayout L;
   L.dy_stride = (uint32_t)((rows * 128 + 1023) & ~1023);
-  L.w_stride = (uint32_t)(((k / 64) * 64 * 128 + 1023) & ~1023);
   L.wt_stride = (uint32_t)((band * 128 + 1023) & ~1023);
   uint32_t off = 0;
   L.dy = off;
   off += ns * L.dy_stride;
-  L.w = off;
-  off += ns * L.w_stride;
   L.wt = off;
   off += ns * L.wt_stride;
   L.bars = off;
@@ -82,13 +81,16 @@ constexpr int kDxThreads = 320;  // producer warp, MMA warp, two sets of 4 densi
 // One CTA owns a feature band, a batch half of up to 256 rows (up to two 128-row
 // TMEM accumulators of NB columns) and a chunk of whole items:
 //   producer (warp 0, one thread): the item's dY tile (the half's rows x 64
-//     labels, K-major) and its weight rows (64 labels x k) into a ring stage;
+//     labels) into a ring stage, and the item's weight rows and index rows into
+//     L2 ahead of use;
 //   densify (two sets of four warps, warps 2-5 for the even items of the chunk,
-//     6-9 for the odd ones; the thread of slot s): clears, for each group of the
-//     item NS back (the previous user of the stage), that group's columns of the
-//     Wt row of slot s's feature, then, after a barrier of its set, writes column
-//     s of each present group's weights into its columns of the row of the
-//     slot's feature when it falls in the band;
+//     6-9 for the odd ones; the thread of slot s): loads column s of each present
+//     group's weights from global memory when the slot's feature falls in the
+//     band (the lanes of a warp read consecutive slots of one weight row), clears,
+//     for each group of the item NS back (the previous user of the stage), that
+//     group's columns of the Wt row of its slot's feature, then, after a barrier
+//     of its set, writes the loaded column into the group's columns of the row
+//     of the slot's feature;
 //   MMA (warp 1): D[t] += dY_u[128t.., labels] . Wt_u^T for each batch tile t;
 //   epilogue (warps 2-9): the TMEM accumulators to the chunk partial.
 // The warps of a set run the same number of iterations (one per item of the
@@ -96,7 +98,7 @@ constexpr int kDxThreads = 320;  // producer warp, MMA warp, two sets of 4 densi
 // abort flag and the remaining iterations skip their work.
 template <int kG, int kK>
 __global__ void __launch_bounds__(kDxThreads, 1)
-    k_dx_band(DxArgs a, const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__ CUtensorMap tm_w) {
+    k_dx_band(DxArgs a, const __grid_constant__ CUtensorMap tm_dy) {
   extern __shared__ __align__(1024) uint8_t smem[];
   constexpr int NG = items_ng(kG);  // groups per item
   constexpr int GB = kG * 2;        // bytes of one group's columns in a 128-byte row
@@ -120,11 +122,10 @@ __global__ void __launch_bounds__(kDxThreads, 1)
   const uint32_t base = align1024(smem_u32(smem));
   uint8_t* gbase = smem + (base - smem_u32(smem));
   auto DYS = [&](int st) -> uint32_t { return base + Lo.dy + st * Lo.dy_stride; };
-  auto WS = [&](int st) -> uint32_t { return base + Lo.w + st * Lo.w_stride; };
   auto WT = [&](int st) -> uint32_t { return base + Lo.wt + st * Lo.wt_stride; };
   uint64_t* bars = reinterpret_cast<uint64_t*>(gbase + Lo.bars);
-  uint64_t* full = bars;                      // [NS] dY tile + weight rows landed (1 + tx bytes)
-  uint64_t* empty = full + kMaxDxStages;      // [NS] both read: MMA commit + 4 densify warps
+  uint64_t* full = bars;                      // [NS] dY tile landed (1 + tx bytes)
+  uint64_t* empty = full + kMaxDxStages;      // [NS] dY tile read (MMA commit)
   uint64_t* wt_full = empty + kMaxDxStages;   // [NS] Wt block written (4 densify warps)
   uint64_t* wt_empty = wt_full + kMaxDxStages;  // [NS] Wt block read by the MMA
   uint64_t* done = wt_empty + kMaxDxStages;     // every MMA of the CTA finished
@@ -135,7 +136,7 @@ __global__ void __launch_bounds__(kDxThreads, 1)
   if (threadIdx.x == 0) {
     for (int st = 0; st < NS; ++st) {
       mbar_init(&full[st], 1);
-      mbar_init(&empty[st], 5);   // MMA commit + the 4 warps of one densify set
+      mbar_init(&empty[st], 1);   // MMA commit
       mbar_init(&wt_full[st], 4);
       mbar_init(&wt_empty[st], 1);
     }
@@ -162,7 +163,7 @@ __global__ void __launch_bounds__(kDxThreads, 1)
   if (w == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      const uint32_t bytes = (uint32_t)(BH + kK) * 128;  // dY tile + weight rows (full boxes)
+      const uint32_t bytes = (uint32_t)BH * 128;  // dY tile (full boxes)
       const int64_t w_elems = sh.L * kK, ix_elems = sh.n_groups * kK;
       // a ring load from HBM takes longer than the ring's MMA work: the tiles of
       // later items are requested into L2 ahead of their ring loads (ranges clamped
@@ -187,9 +188,6 @@ __global__ void __launch_bounds__(kDxThreads, 1)
                         &full[st]);
         } else
           tma_load_2d(DYS(st), &tm_dy, (int)(sg * kItemLabels), 256 * bh, &full[st]);
-#pragma unroll
-        for (int blk = 0; blk < kK / 64; ++blk)
-          tma_load_2d(WS(st) + (uint32_t)(blk * 64 * 128), &tm_w, 64 * blk, (int)(sg * kItemLabels), &full[st]);
         if (++st == NS) {
           st = 0;
           ph ^= 1;
@@ -240,10 +238,7 @@ __global__ void __launch_bounds__(kDxThreads, 1)
     const int set = (w - 2) >> 2;          // items i = set, set + 2, ...
     const int s = (threadIdx.x - 64) & 127;  // this thread's slot
     const bool slot_ok = s < kK;
-    // column s of the weight rows: 64-slot block s/64, 16-byte chunk (s%64)/8 of
-    // each 128-byte row (TMA 128-byte swizzle), element s%8
-    const uint32_t wcol = (uint32_t)((s >> 6) * 64 * 128 + (s & 7) * 2);
-    const uint32_t wchunk = (uint32_t)((s & 63) >> 3);
+    const uint16_t* wbits = reinterpret_cast<const uint16_t*>(a.W);
     // the slot's feature in group j of item i, relative to the band (-1 if absent)
     auto feat = [&](int i, int j) -> int {
       if (!slot_ok || i < 0 || i >= n || j >= cnt(i)) return -1;
@@ -277,6 +272,18 @@ __global__ void __launch_bounds__(kDxThreads, 1)
         ob[j] = oc[j];
         oc[j] = feat(i + 6 - NS, j);
       }
+      // column s of the item's weights (label rows 64 (u0 + i) + j G + l), loaded
+      // before the waits so that their latency hides behind them
+      uint32_t pk[NG][kG / 2];
+#pragma unroll
+      for (int j = 0; j < NG; ++j) {
+        if (fcur[j] >= 0 && fcur[j] < nf) {
+          const uint16_t* col = wbits + ((u0 + i) * kItemLabels + j * kG) * kK + s;
+#pragma unroll
+          for (int l = 0; l < kG; l += 2)
+            pk[j][l / 2] = (uint32_t)__ldg(col + (int64_t)l * kK) | ((uint32_t)__ldg(col + (int64_t)(l + 1) * kK) << 16);
+        }
+      }
       uint8_t* wt = gbase + Lo.wt + st * Lo.wt_stride;
       // the MMA of item i - NS has read this stage's Wt block: clear its groups' columns
       const bool ok = __all_sync(0xffffffffu, wait_or_abort(&wt_empty[st], ph ^ 1u, abort_flag));
@@ -293,33 +300,20 @@ __global__ void __launch_bounds__(kDxThreads, 1)
       // every old column run is clear before any new one is written (slots of
       // different items may share a feature)
       named_bar(1 + set, 128);
-      const bool ok2 = ok && __all_sync(0xffffffffu, wait_or_abort(&full[st], ph, abort_flag));
-      if (ok2) {
-        const uint8_t* wst = gbase + Lo.w + st * Lo.w_stride + wcol;
+      if (ok) {
 #pragma unroll
         for (int j = 0; j < NG; ++j) {
           const int f = fcur[j];
           if (f < 0 || f >= nf) continue;
-          uint32_t pk[kG / 2];
-#pragma unroll
-          for (int l = 0; l < kG; l += 2) {
-            const int r0 = j * kG + l, r1 = r0 + 1;  // weight rows (labels) of the item
-            const uint32_t lo = *reinterpret_cast<const uint16_t*>(wst + r0 * 128 + ((wchunk ^ (r0 & 7)) << 4));
-            const uint32_t hi = *reinterpret_cast<const uint16_t*>(wst + r1 * 128 + ((wchunk ^ (r1 & 7)) << 4));
-            pk[l / 2] = lo | (hi << 16);
-          }
 #pragma unroll
           for (int cc = 0; cc < GB / 16; ++cc)
             *reinterpret_cast<uint4*>(wt + sw128((uint32_t)(f * 128 + j * GB + cc * 16))) =
-                make_uint4(pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
+                make_uint4(pk[j][4 * cc], pk[j][4 * cc + 1], pk[j][4 * cc + 2], pk[j][4 * cc + 3]);
         }
         fence_proxy_async_smem();
       }
       __syncwarp();
-      if (lane == 0 && ok2) {
-        mbar_arrive(&empty[st]);
-        mbar_arrive(&wt_full[st]);
-      }
+      if (lane == 0 && ok) mbar_arrive(&wt_full[st]);
       if ((st += 2) >= NS) {
         st -= NS;
         ph ^= 1u;
@@ -392,22 +386,22 @@ int64_t dx_items(int64_t n_groups, int G) { return v2::n_items_of(n_groups, G); 
 // outside the tensor and read as zeros).
 template <int kG, int kK>
 cudaError_t launch_dx_t(v2::DxArgs a, const void* dY, const void* W, cudaStream_t st) {
+  (void)W;  // the densify warps read a.W directly
   const int rows = a.sh.Bp < 256 ? a.sh.Bp : 256;
   const size_t smem = dx_smem(rows, a.band, kK, a.ns);
   auto kern = v2::k_dx_band<kG, kK>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  CUtensorMap tm_dy, tm_w;
+  CUtensorMap tm_dy;
   if (a.group_major)
     e = tmap_2d(&tm_dy, dY, (uint64_t)a.sh.Bp, (uint64_t)dx_items(a.sh.n_groups, kG) * v2::kItemLabels,
                 (uint64_t)a.sh.Bp * 2, 64, v2::kItemLabels);
   else
     e = tmap_2d(&tm_dy, dY, (uint64_t)a.sh.L, (uint64_t)a.sh.B, (uint64_t)a.sh.L * 2, v2::kItemLabels,
                 (uint32_t)rows);
-  if (e == cudaSuccess) e = tmap_2d(&tm_w, W, kK, (uint64_t)a.sh.L, (uint64_t)kK * 2, 64, v2::kItemLabels);
   if (e != cudaSuccess) return e;
   const int grid = a.n_bands * a.n_halves * a.n_chunks;
-  kern<<<grid, v2::kDxThreads, smem, st>>>(a, tm_dy, tm_w);
+  kern<<<grid, v2::kDxThreads, smem, st>>>(a, tm_dy);
   return cudaGetLastError();
 }
 
