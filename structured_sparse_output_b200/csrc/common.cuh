@@ -171,6 +171,11 @@ __device__ __forceinline__ bool named_bar_or(int id, int nthreads, bool pred) {
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+// Wait until at most N of this thread's committed cp.async groups are pending.
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
 // Make generic-proxy shared-memory writes visible to the tensor core (async proxy).
 // The mbarrier receives one arrival once every cp.async this thread issued so
 // far has landed (the barrier's expected count includes this arrival).

@@ -78,15 +78,19 @@ __device__ __forceinline__ uint64_t operand_desc(uint32_t s, int kk, int BK) {
   }
 }
 
-template <typename T, bool kAMN, bool kBMN, int kEpi, int kBN>
+template <typename T, bool kAMN, bool kBMN, int kEpi, int kBN, int kStages>
 __global__ void __launch_bounds__(kGThreads, 1) k_gemm(GemmArgs a) {
   extern __shared__ __align__(1024) uint8_t smem[];
   constexpr int R = 128 / sizeof(T), KI = Elem<T>::kMmaK;
   constexpr int BK = 2 * R;  // two 128B rows of K per stage
+  // kStages = 2: the operands of K chunk i+1 load while the MMAs of chunk i run
+  // (for grids that leave SMs idle); kStages = 1: several CTAs share an SM and
+  // overlap each other
+  constexpr uint32_t kStageA = (uint32_t)kBM * BK * sizeof(T), kStageB = (uint32_t)kBN * BK * sizeof(T);
   const uint32_t base = align1024(smem_u32(smem));
-  const uint32_t sa = base;
-  const uint32_t sb = sa + (uint32_t)kBM * BK * sizeof(T);
-  uint8_t* gen = smem + (sb + (uint32_t)kBN * BK * sizeof(T) - smem_u32(smem));
+  auto SA = [&](int st) -> uint32_t { return base + (uint32_t)st * (kStageA + kStageB); };
+  auto SB = [&](int st) -> uint32_t { return SA(st) + kStageA; };
+  uint8_t* gen = smem + (base + kStages * (kStageA + kStageB) - smem_u32(smem));
   uint64_t* bar = reinterpret_cast<uint64_t*>(gen);
   uint32_t* tslot = reinterpret_cast<uint32_t*>(bar + 1);
   int* abort_flag = reinterpret_cast<int*>(tslot + 1);
@@ -115,30 +119,67 @@ __global__ void __launch_bounds__(kGThreads, 1) k_gemm(GemmArgs a) {
   const T* Bm = static_cast<const T*>(a.Bm);
   bool ok = true;
 
-  for (int k0 = k_begin; k0 < k_end; k0 += BK) {
-    load_operand<T, kAMN>(sa, A, a.lda, a.M, k_end, m0, k0, BK);
-    load_operand<T, kBMN, kBN>(sb, Bm, a.ldb, a.N, k_end, n0, k0, BK);
+  auto load = [&](int k0, int st) {
+    load_operand<T, kAMN>(SA(st), A, a.lda, a.M, k_end, m0, k0, BK);
+    load_operand<T, kBMN, kBN>(SB(st), Bm, a.ldb, a.N, k_end, n0, k0, BK);
     cp_async_commit();
-    cp_async_wait_all();
+  };
+  const int n_chunks = k_end > k_begin ? (k_end - k_begin + BK - 1) / BK : 0;
+  if (kStages == 2 && n_chunks > 0) load(k_begin, 0);
+  for (int it = 0; it < n_chunks; ++it) {
+    const int st = kStages == 2 ? (it & 1) : 0;
+    if constexpr (kStages == 1) {
+      // the stage was read by the MMAs of chunk it-1
+      if (it >= 1) {
+        const bool w = mbar_wait(bar, phase);
+        phase ^= 1u;
+        if (!w) *abort_flag = 1;
+      }
+      load(k_begin + it * BK, 0);
+      cp_async_wait_all();
+    } else if (it + 1 < n_chunks) {
+      // the other stage was read by the MMAs of chunk it-1: wait for them, then load chunk it+1 into it
+      if (it >= 1) {
+        const bool w = mbar_wait(bar, phase);
+        phase ^= 1u;
+        if (!w) *abort_flag = 1;
+      }
+      load(k_begin + (it + 1) * BK, st ^ 1);
+      cp_async_wait_group<1>();  // chunk it has landed
+    } else {
+      if (it >= 1) {
+        const bool w = mbar_wait(bar, phase);
+        phase ^= 1u;
+        if (!w) *abort_flag = 1;
+      }
+      cp_async_wait_all();
+    }
     fence_proxy_async_smem();
+    tc_fence_before();
     __syncthreads();
+    tc_fence_after();
+    if (*abort_flag) {
+      ok = false;
+      break;
+    }
     if (threadIdx.x == 0) {
-      tc_fence_after();
+      const uint32_t sa = SA(st), sb = SB(st);
       for (int kk = 0; kk < BK / KI; ++kk)
         mma_ss<Elem<T>::kTF32>(tmem, operand_desc<T, kAMN>(sa, kk, BK), operand_desc<T, kBMN, kBN>(sb, kk, BK), idesc,
-                               (k0 > k_begin || kk > 0) ? 1u : 0u);
+                               (it > 0 || kk > 0) ? 1u : 0u);
       mma_commit(bar);
     }
+  }
+  // the MMAs of the last chunk
+  if (ok && n_chunks > 0) {
     const bool w = mbar_wait(bar, phase);
     phase ^= 1u;
     if (!w) *abort_flag = 1;
     tc_fence_after();
     __syncthreads();
-    if (*abort_flag) {
-      ok = false;
-      break;
-    }
+    if (*abort_flag) ok = false;
   }
+  cp_async_wait_all();
 
   const int m = m0 + threadIdx.x;
   const uint32_t lane = tmem + (((threadIdx.x / 32) * 32u) << 16);
@@ -226,16 +267,27 @@ __global__ void k_split_reduce(const float* __restrict__ P, float* __restrict__ 
   }
 }
 
-template <typename T, bool kAMN, bool kBMN, int kEpi, int kBN = 128>
-cudaError_t run_gemm(const GemmArgs& a, int splits, cudaStream_t st) {
+template <typename T, bool kAMN, bool kBMN, int kEpi, int kBN, int kStages>
+cudaError_t run_gemm_t(const GemmArgs& a, dim3 grid, cudaStream_t st) {
   constexpr int BK = 2 * (128 / (int)sizeof(T));
-  const size_t smem = 1024 + (size_t)(kBM + kBN) * BK * sizeof(T) + 64;
-  auto kern = k_gemm<T, kAMN, kBMN, kEpi, kBN>;
+  const size_t smem = 1024 + kStages * (size_t)(kBM + kBN) * BK * sizeof(T) + 64;
+  auto kern = k_gemm<T, kAMN, kBMN, kEpi, kBN, kStages>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  dim3 grid((a.M + kBM - 1) / kBM, (a.N + kBN - 1) / kBN, splits);
   kern<<<grid, kGThreads, smem, st>>>(a);
   return cudaGetLastError();
+}
+
+// Two stages when the grid leaves SMs without a CTA, one (several CTAs per SM)
+// otherwise.
+template <typename T, bool kAMN, bool kBMN, int kEpi, int kBN = 128>
+cudaError_t run_gemm(const GemmArgs& a, int splits, cudaStream_t st) {
+  const dim3 grid((a.M + kBM - 1) / kBM, (a.N + kBN - 1) / kBN, splits);
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    sms = 0;
+  if ((int64_t)grid.x * grid.y * grid.z <= sms) return run_gemm_t<T, kAMN, kBMN, kEpi, kBN, 2>(a, grid, st);
+  return run_gemm_t<T, kAMN, kBMN, kEpi, kBN, 1>(a, grid, st);
 }
 
 }  // namespace
