@@ -8,9 +8,11 @@
 // or every slot (dW: N = k):
 //   forward  logits_g^T [MW, Bp] = W_g [MW, k] . Xg^T     (K = k)
 //   dW       dW_g^T     [MW, k]  = dY_g^T [MW, Bp] . Xg   (K = Bp)
-//   warp 0     MMA issuer (one thread): issues each group's forward and dW
-//              product as soon as its inputs are ready;
-//   producers  six warps (three for G = 64): the gather-once tile Xg = X[:, I_g]
+//   warps 0, 12  MMA issuers (one thread each): warp 0 issues each group's
+//              forward, warp 12 its dW product, each as soon as its inputs are
+//              ready (in the narrow block of the G = 64 update kernels warp 0
+//              issues both);
+//   producers  six warps (three in the narrow block): the gather-once tile Xg = X[:, I_g]
 //              (k rows of X^T) and the G x k weight block, staged with cp.async
 //              into a 2-stage ring (all of them fill the stage of each group);
 //   epilogue   eight warps: each thread owns one label and a run of batch rows of the
@@ -113,39 +115,46 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
 
 // ============================================================ k_step2
 // Warp roles (warp w runs on scheduler w % 4, which also fixes the TMEM lane
-// quarter an epilogue warp can read).  The MMA issuer (warp 0) shares its
-// scheduler with no producer: the producers' stream of cp.async fills the
-// memory-instruction queue of theirs, and each barrier test of the issuer would
+// quarter an epilogue warp can read).  The MMA issuers (warps 0 and 12) share
+// their scheduler with no producer: the producers' stream of cp.async fills the
+// memory-instruction queue of theirs, and each barrier test of an issuer would
 // wait behind it.
-//   G <= 32: six producer warps (1-3, 5-7, two on each of schedulers 1-3) keep
-//            more gathered rows in flight; epilogue warps 4 and 8 (quarter 0), 9
-//            and 13 (1), 10 and 14 (2), 11 and 15 (3); warp 12 idles.  512 threads.
-//   G = 64:  three producer warps (1-3) and epilogue warps 4-11, 384 threads: the
-//            64-label epilogue needs the registers of the smaller block.
-constexpr int kStepMma = 0;        // warp id of the MMA issuer
+//   wide block (512 threads): warp 0 issues the forwards, warp 12 the dW
+//            products; six producer warps (1-3, 5-7, two on each of schedulers
+//            1-3) keep more gathered rows in flight; epilogue warps 4 and 8
+//            (quarter 0), 9 and 13 (1), 10 and 14 (2), 11 and 15 (3).
+//   narrow block (384 threads, G = 64 with the SGD update, whose epilogue needs
+//            the registers): warp 0 issues both kinds, three producer warps
+//            (1-3), epilogue warps 4-11.
+constexpr int kStepMma = 0;        // warp id of the forward issuer
+constexpr int kStepMmaW = 12;      // warp id of the dW issuer
 constexpr int kStepEpi = 8;        // epilogue warps: 4 lane quarters x 2 column halves
 constexpr int kStepEpiThreads = 32 * kStepEpi;
-__host__ __device__ constexpr int step_prod_warps(int G) { return G == 64 ? 3 : 6; }
-__host__ __device__ constexpr int step_threads(int G) { return G == 64 ? 32 * 12 : 32 * 16; }
+// The wide block (16 warps) for every kernel but the G = 64 update kernels, whose
+// 64-label epilogue with the SGD update needs the registers of a 12-warp block.
+__host__ __device__ constexpr bool step_wide(int G, int upd) { return !(G == 64 && upd > 0); }
+__host__ __device__ constexpr int step_prod_warps(bool wide) { return wide ? 6 : 3; }
+__host__ __device__ constexpr int step_threads(bool wide) { return wide ? 32 * 16 : 32 * 12; }
 // producer index of warp w (-1: not a producer)
-template <int kG>
+template <bool kWide>
 __device__ __forceinline__ int step_prod_part(int w) {
-  if constexpr (kG == 64) return w >= 1 && w <= 3 ? w - 1 : -1;
-  else return w >= 1 && w <= 3 ? w - 1 : w >= 5 && w <= 7 ? w - 2 : -1;
+  if constexpr (kWide) return w >= 1 && w <= 3 ? w - 1 : w >= 5 && w <= 7 ? w - 2 : -1;
+  else return w >= 1 && w <= 3 ? w - 1 : -1;
 }
 // epilogue index ew = quarter + 4 * half of warp w (-1: not an epilogue warp)
-template <int kG>
+template <bool kWide>
 __device__ __forceinline__ int step_epi_index(int w) {
-  if constexpr (kG == 64) return w >= 4 && w <= 11 ? w - 4 : -1;
-  else return w == 4 ? 0 : w == 8 ? 4 : w >= 9 && w != 12 ? w - 8 : -1;
+  if constexpr (kWide) return w == 4 ? 0 : w == 8 ? 4 : w >= 9 && w != 12 ? w - 8 : -1;
+  else return w >= 4 && w <= 11 ? w - 4 : -1;
 }
 
 template <int kG, int kK, int kUpd>
-__global__ void __launch_bounds__(step_threads(kG), 1)
+__global__ void __launch_bounds__(step_threads(step_wide(kG, kUpd)), 1)
     k_step2(StepArgs a, const __nv_bfloat16* __restrict__ Xt, const __nv_bfloat16* __restrict__ W,
             const __grid_constant__ CUtensorMap tm_dy) {
   extern __shared__ __align__(1024) uint8_t smem[];
   constexpr int MW = step_mw(kG);     // rows of the weight-stationary MMAs
+  constexpr bool kWide = step_wide(kG, kUpd);
   constexpr int NGI = 64 / kG;        // groups per 64-label item of the gradient buffer
   const TailShape sh = a.sh;
   const int Bp = sh.Bp;
@@ -167,15 +176,24 @@ __global__ void __launch_bounds__(step_threads(kG), 1)
   const int w = warp_id(), lane = lane_id();
   if (threadIdx.x == 0) {
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&full[s], 32 * step_prod_warps(kG));
+      mbar_init(&full[s], 32 * step_prod_warps(kWide));
       mbar_init(&empty[s], 1);
       mbar_init(&fwd_full[s], 1);
       mbar_init(&dy_full[s], kStepEpi);
       mbar_init(&dw_full[s], 1);
       mbar_init(&tmem_empty[s], kStepEpi);
     }
-    mbar_init(done, 1);
-    *abort_flag = 0;
+    mbar_init(done, kWide ? 2 : 1);
+    // A limit below one sleep, set only to exercise the abort paths, makes the
+    // first wait of every warp run out at once (the waits themselves read the
+    // limit only after their first, blocking test: a short limit would not make a
+    // wait whose phase completes within that test run out).
+    if (g_wait_limit_ns < kWaitSuspendNs) {
+      *abort_flag = 1;
+      record_error(kErrTimeout);
+    } else {
+      *abort_flag = 0;
+    }
     fence_mbar_init();
   }
   // TMEM: logits^T accumulators F[2] (Bp columns over the lane quarters: Bp/4 for
@@ -202,17 +220,17 @@ __global__ void __launch_bounds__(step_threads(kG), 1)
   const int64_t ge = (int64_t)(blockIdx.x + 1) * sh.n_groups / gridDim.x;
   const int n_items = (int)(ge - gb);
 
-  if (step_prod_part<kG>(w) >= 0) {
+  if (step_prod_part<kWide>(w) >= 0) {
     // ------------------------------------------------- cp.async producers
     // the producer warps fill the stage of every item i (stage i & 1); warp part
     // copies the groups of four rows part, part + P, ...  Lane (rg, sub) copies
     // the 16-byte chunk sub of every 128-byte segment of its rows, so that 8
     // consecutive lanes read one segment; the feature indices of its rows sit in
     // registers.
-    constexpr int P = step_prod_warps(kG);
+    constexpr int P = step_prod_warps(kWide);
     constexpr int kQuads = kK / 4;                 // groups of four rows
     constexpr int kRows = (kQuads + P - 1) / P;    // per warp (the last may be short)
-    const int part = step_prod_part<kG>(w), ht = lane;
+    const int part = step_prod_part<kWide>(w), ht = lane;
     const int sub = ht & 7, rg = ht >> 3;
     for (int i = 0; i < n_items; ++i) {
       const int64_t g = gb + i;
@@ -257,58 +275,49 @@ __global__ void __launch_bounds__(step_threads(kG), 1)
       publish_all(&full[half]);
     }
     cp_async_wait_all();
-  } else if (w == kStepMma) {
-    // ------------------------------------------------------------ MMA issuer
-    // Forwards and dW products are issued as their inputs become ready, not in a
-    // fixed interleave: fwd(j) needs its gathered stage (full) and F(j&1) free,
-    // which holds once dW(j-2) was issued (its BCE had finished reading F);
-    // dW(j) needs the BCE of j (dy_full) and D(j&1) read out for j-2
-    // (tmem_empty).  Lane 0 polls; the decisions are broadcast so the warp stays
-    // converged.  No progress for the wait limit raises the abort flag.
-    //   forward: A = W_g (K-major, label rows), B = Xg (MN-major: batch
-    //            contiguous, 64-column blocks kK*128 bytes apart), K = 16 slots;
-    //   dW:      A = dY^T (K-major, label rows), B = Xg (K-major: slot rows),
-    //            K = 16 batch rows.
-    const uint32_t idesc_f = make_idesc(1, 0, 1, MW, (uint32_t)Bp);
-    const uint32_t idesc_w = make_idesc(1, 0, 0, MW, kK);
-    int nf = 0, nd = 0;
-    // the timer is read only while nothing is ready (a read costs hundreds of
-    // cycles): t_idle is when the current idle stretch began, 0 after progress
-    uint64_t t_idle = 0;
-    const uint64_t limit = g_wait_limit_ns;
-    while (nd < n_items) {
-      bool did = false;
-      if (nf < n_items && nf <= nd + 1) {
-        const int s = nf & 1;
-        const bool rdy = __shfl_sync(0xffffffffu, lane == 0 ? mbar_test_wait(&full[s], (nf >> 1) & 1) : false, 0);
-        if (rdy) {
+  } else if (w == kStepMma || (kWide && w == kStepMmaW)) {
+    // ------------------------------------------------------------ MMA issuers
+    // Wide block: two warps, each sleeping in the barrier it waits for (no polling
+    // loop over both kinds, so each wakes as soon as its operands are ready; on the
+    // step of 670K labels this is 6% faster), one thread of each issuing:
+    //   warp kStepMma:  forward of group i once its stage is loaded (full) and
+    //                   F(i&1) is free (the BCE of group i - 2 has read it:
+    //                   dy_full).  A = W_g (K-major, label rows), B = Xg
+    //                   (MN-major: batch contiguous, 64-column blocks kK*128
+    //                   bytes apart), K = 16 slots;
+    //   warp kStepMmaW: dW of group i once its BCE is done (dy_full) and D(i&1)
+    //                   has been read out for group i - 2 (tmem_empty).
+    //                   A = dY^T (K-major, label rows), B = Xg (K-major: slot
+    //                   rows), K = 16 batch rows; its commits free the readout
+    //                   (dw_full) and the stage (empty).
+    // A wait that runs out raises the abort flag; the other waits then fail fast.
+    // Descriptors advance by constant start-address offsets (16-byte units).
+    if constexpr (kWide) {
+      if (w == kStepMma) {
+        const uint32_t idesc_f = make_idesc(1, 0, 1, MW, (uint32_t)Bp);
+        for (int i = 0; i < n_items; ++i) {
+          const int s = i & 1;
+          if (!__all_sync(0xffffffffu, wait_or_abort(&full[s], (i >> 1) & 1, abort_flag))) break;
+          if (i >= 2 && !__all_sync(0xffffffffu, wait_or_abort(&dy_full[s], ((i - 2) >> 1) & 1, abort_flag))) break;
           if (lane == 0) {
             tc_fence_after();
-            // descriptors advance by constant start-address offsets (16-byte units):
-            // the issuing warp shares its scheduler with busy warps, so each MMA
-            // costs only a few instructions
             const uint64_t ad0 = make_sdesc(WG(s), 16, 1024, kLayoutSw128);
             const uint64_t bd0 = make_sdesc(XG(s), (uint32_t)kK * 128, 1024, kLayoutSw128);
             const uint32_t f = F(s);
 #pragma unroll
             for (int kk = 0; kk < kK / 16; ++kk)
-              mma_ws(f, ad0 + (uint64_t)(((kk / 4) * MW * 128 + (kk % 4) * 32) >> 4), bd0 + (uint64_t)(kk * 128), idesc_f,
-                     kk > 0 ? 1u : 0u);
+              mma_ws(f, ad0 + (uint64_t)(((kk / 4) * MW * 128 + (kk % 4) * 32) >> 4), bd0 + (uint64_t)(kk * 128),
+                     idesc_f, kk > 0 ? 1u : 0u);
             mma_commit(&fwd_full[s]);
           }
           __syncwarp();
-          ++nf;
-          did = true;
         }
-      }
-      if (nd < nf) {
-        const int s = nd & 1;
-        const bool rdy = __shfl_sync(0xffffffffu,
-                                     lane == 0 ? (mbar_test_wait(&dy_full[s], (nd >> 1) & 1) &&
-                                                  mbar_test_wait(&tmem_empty[s], ((nd >> 1) & 1) ^ 1))
-                                               : false,
-                                     0);
-        if (rdy) {
+      } else {
+        const uint32_t idesc_w = make_idesc(1, 0, 0, MW, kK);
+        for (int i = 0; i < n_items; ++i) {
+          const int s = i & 1;
+          if (!__all_sync(0xffffffffu, wait_or_abort(&dy_full[s], (i >> 1) & 1, abort_flag))) break;
+          if (!__all_sync(0xffffffffu, wait_or_abort(&tmem_empty[s], ((i >> 1) & 1) ^ 1, abort_flag))) break;
           if (lane == 0) {
             tc_fence_after();
             const uint64_t ad0 = make_sdesc(base + DY(s), 16, 1024, kLayoutSw128);
@@ -329,37 +338,117 @@ __global__ void __launch_bounds__(step_threads(kG), 1)
             mma_commit(&empty[s]);
           }
           __syncwarp();
-          ++nd;
-          did = true;
         }
       }
-      if (did) {
-        t_idle = 0;
-      } else {
-        if (*abort_flag) break;
-        const uint64_t now = globaltimer_ns();
-        if (t_idle == 0) t_idle = now;
-        if (now - t_idle > limit) {
-          if (lane == 0) {
-            *abort_flag = 1;
-            record_error(kErrTimeout);
+    } else {
+      // Narrow block: warp 0 issues both kinds.
+      // Forwards and dW products are issued as their inputs become ready, not in a
+      // fixed interleave: fwd(j) needs its gathered stage (full) and F(j&1) free,
+      // which holds once dW(j-2) was issued (its BCE had finished reading F);
+      // dW(j) needs the BCE of j (dy_full) and D(j&1) read out for j-2
+      // (tmem_empty).  Lane 0 polls; the decisions are broadcast so the warp stays
+      // converged.  No progress for the wait limit raises the abort flag.
+      //   forward: A = W_g (K-major, label rows), B = Xg (MN-major: batch
+      //            contiguous, 64-column blocks kK*128 bytes apart), K = 16 slots;
+      //   dW:      A = dY^T (K-major, label rows), B = Xg (K-major: slot rows),
+      //            K = 16 batch rows.
+      const uint32_t idesc_f = make_idesc(1, 0, 1, MW, (uint32_t)Bp);
+      const uint32_t idesc_w = make_idesc(1, 0, 0, MW, kK);
+      int nf = 0, nd = 0;
+      // the timer is read only while nothing is ready, and then once every 64 polls
+      // (a read costs hundreds of cycles, which would delay the next issue): t_idle
+      // is when the current idle stretch began, 0 after progress
+      uint64_t t_idle = 0;
+      uint32_t idle_polls = 0;
+      const uint64_t limit = g_wait_limit_ns;
+      while (nd < n_items) {
+        bool did = false;
+        if (nf < n_items && nf <= nd + 1) {
+          const int s = nf & 1;
+          const bool rdy = __shfl_sync(0xffffffffu, lane == 0 ? mbar_test_wait(&full[s], (nf >> 1) & 1) : false, 0);
+          if (rdy) {
+            if (lane == 0) {
+              tc_fence_after();
+              // descriptors advance by constant start-address offsets (16-byte units):
+              // the issuing warp shares its scheduler with busy warps, so each MMA
+              // costs only a few instructions
+              const uint64_t ad0 = make_sdesc(WG(s), 16, 1024, kLayoutSw128);
+              const uint64_t bd0 = make_sdesc(XG(s), (uint32_t)kK * 128, 1024, kLayoutSw128);
+              const uint32_t f = F(s);
+#pragma unroll
+              for (int kk = 0; kk < kK / 16; ++kk)
+                mma_ws(f, ad0 + (uint64_t)(((kk / 4) * MW * 128 + (kk % 4) * 32) >> 4), bd0 + (uint64_t)(kk * 128), idesc_f,
+                       kk > 0 ? 1u : 0u);
+              mma_commit(&fwd_full[s]);
+            }
+            __syncwarp();
+            ++nf;
+            did = true;
           }
-          __syncwarp();
-          break;
         }
-        // no sleep here: a suspended issuer wakes far later than the barriers
-        // complete, and the tensor core would wait for it
+        if (nd < nf) {
+          const int s = nd & 1;
+          const bool rdy = __shfl_sync(0xffffffffu,
+                                       lane == 0 ? (mbar_test_wait(&dy_full[s], (nd >> 1) & 1) &&
+                                                    mbar_test_wait(&tmem_empty[s], ((nd >> 1) & 1) ^ 1))
+                                                 : false,
+                                       0);
+          if (rdy) {
+            if (lane == 0) {
+              tc_fence_after();
+              const uint64_t ad0 = make_sdesc(base + DY(s), 16, 1024, kLayoutSw128);
+              const uint64_t bd0 = make_sdesc(XG(s), 16, 1024, kLayoutSw128);
+              const uint32_t d = D(s);
+              auto dw_mma = [&](int kk) {
+                mma_ws(d, ad0 + (uint64_t)(((kk / 4) * MW * 128 + (kk % 4) * 32) >> 4),
+                       bd0 + (uint64_t)(((kk / 4) * kK * 128 + (kk % 4) * 32) >> 4), idesc_w, kk > 0 ? 1u : 0u);
+              };
+              if (Bp == 256) {
+#pragma unroll
+                for (int kk = 0; kk < 16; ++kk) dw_mma(kk);
+              } else {
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) dw_mma(kk);
+              }
+              mma_commit(&dw_full[s]);
+              mma_commit(&empty[s]);
+            }
+            __syncwarp();
+            ++nd;
+            did = true;
+          }
+        }
+        if (did) {
+          t_idle = 0;
+          idle_polls = 0;
+        } else {
+          if (*abort_flag) break;
+          if ((idle_polls++ & 63u) == 0) {
+            const uint64_t now = globaltimer_ns();
+            if (t_idle == 0) t_idle = now;
+            if (now - t_idle > limit) {
+              if (lane == 0) {
+                *abort_flag = 1;
+                record_error(kErrTimeout);
+              }
+              __syncwarp();
+              break;
+            }
+          }
+          // no sleep here: a suspended issuer wakes far later than the barriers
+          // complete, and the tensor core would wait for it
+        }
       }
     }
-    // Also after an abort: the CTA frees TMEM and exits only once every MMA it
-    // issued has finished writing TMEM and reading shared memory.
+    // Also after an abort: the CTA frees TMEM and exits only once every MMA its
+    // issuers issued has finished writing TMEM and reading shared memory.
     if (lane == 0) mma_commit(done);
     __syncwarp();
     (void)__all_sync(0xffffffffu, mbar_wait(done, 0));
-  } else if (step_epi_index<kG>(w) >= 0) {
+  } else if (step_epi_index<kWide>(w) >= 0) {
     // ------------------------------------------------------------- epilogue
     // warp (q, hh): TMEM lane quarter q, half hh of the quarter's columns
-    const int ew = step_epi_index<kG>(w), q = w & 3, hh = ew >> 2;
+    const int ew = step_epi_index<kWide>(w), q = w & 3, hh = ew >> 2;
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     // this thread's label m (a row of the MW-row products), its run of nct batch
     // rows from b0 (logits) and of NSL slots from s0 (dW)
@@ -633,7 +722,7 @@ cudaError_t launch_step_t(const v2::StepArgs& a, int grid, const void* Xt, const
   const uint64_t n_items = (uint64_t)(a.sh.n_groups + 64 / kG - 1) / (64 / kG);
   e = tmap_2d(&tm_dy, a.dY_out, (uint64_t)a.sh.Bp, n_items * 64, (uint64_t)a.sh.Bp * 2, 64, kG);
   if (e != cudaSuccess) return e;
-  kern<<<grid, v2::step_threads(kG), smem, st>>>(a, static_cast<const __nv_bfloat16*>(Xt),
+  kern<<<grid, v2::step_threads(v2::step_wide(kG, kUpd)), smem, st>>>(a, static_cast<const __nv_bfloat16*>(Xt),
                                              static_cast<const __nv_bfloat16*>(W), tm_dy);
   return cudaGetLastError();
 }

@@ -255,11 +255,12 @@ def test_bounded_wait_timeout_is_reported_and_context_survives():
 
 
 def test_short_wait_limit_reaches_the_abort_paths_and_the_context_survives():
-    """A 1 ns limit on the pipelined kernels' inter-warp waits makes the first wait
-    of the step kernel, the dX band kernel and the top-k kernel run out, so each
-    takes its abort path (raise the CTA's abort flag, drain its own copies, commit
-    and wait for its issued MMAs, free TMEM).  The timeout is reported once; with
-    the default limit restored, the same calls give the oracle's results."""
+    """A 1 ns limit on the pipelined kernels' inter-warp waits makes the step
+    kernel's first wait of every warp run out at once (a limit below one sleep
+    raises the CTA's abort flag at the start), and the top-k kernel's first wait
+    that has to sleep, so that each takes its abort path (drain its own copies,
+    commit and wait for its issued MMAs, free TMEM).  The timeout is reported once;
+    with the default limit restored, the same calls give the oracle's results."""
     c = dict(B=256, d=768, n_groups=300, G=32, k=128, dtype="bf16", H=0, p=5)
     idx, X, W, tpos, _ = _step_inputs(c)
     plan = H.haste_plan(idx, c["G"], c["d"])
