@@ -86,10 +86,10 @@ def algorithmic(wl):
 # kernel from one ncu capture (summaries under profiles/), valid only for the
 # source file it was taken on: (config, timed region) -> (bytes, source digest).
 TRAFFIC = {
-    ("670k", "tail_step"): (644.9e6, "c57c4654ec08eb3f"),
-    ("670k", "tail_dx"): (530.1e6, "2115c55101e00c65"),
-    ("8.6m", "tail_step"): (8.83e9, "c57c4654ec08eb3f"),
-    ("8.6m", "tail_dx"): (6.81e9, "2115c55101e00c65"),
+    ("670k", "tail_step"): (645.5e6, "d22391d4777a5228"),
+    ("670k", "tail_dx"): (538.5e6, "09ba676f0abb371c"),
+    ("8.6m", "tail_step"): (8.83e9, "d22391d4777a5228"),
+    ("8.6m", "tail_dx"): (7.01e9, "09ba676f0abb371c"),
     ("670k", "topk_score"): (187.0e6, "48974329ba8749cd"),
 }
 # timed region -> (source file under csrc/, kernel name in the ncu summaries)
