@@ -127,6 +127,8 @@ STEP_CASES = [
     dict(B=37, d=256, n_groups=1, G=32, k=64, dtype="bf16", H=0, p=2),      # a single group
     dict(B=200, d=384, n_groups=301, G=16, k=128, dtype="bf16", H=0, p=6),  # CTA pairs, G = 16
     dict(B=256, d=512, n_groups=5, G=32, k=128, dtype="bf16", H=0, p=4),    # fewer groups than CTA pairs
+    dict(B=200, d=512, n_groups=151, G=64, k=64, dtype="bf16", H=0, p=6),   # G = 64, k = 64, ragged batch
+    dict(B=90, d=384, n_groups=3, G=64, k=128, dtype="bf16", H=0, p=3),     # G = 64, fewer groups than SMs
 ]
 
 
