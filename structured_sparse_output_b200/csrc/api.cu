@@ -833,6 +833,7 @@ haste_status_t bce_step_impl(haste_plan_t p, int32_t B, haste_dtype_t dt, const 
       sa.sh = a.sh;
       sa.idx = p->idx_d;
       sa.dW = static_cast<__nv_bfloat16*>(dW);
+      sa.dw_v8 = (reinterpret_cast<uintptr_t>(dW) & 31) == 0;
       sa.dY_out = static_cast<__nv_bfloat16*>(a.dY_out);
       sa.loss_part = a.loss_part;
       sa.pos_ptr = pos.row_ptr;

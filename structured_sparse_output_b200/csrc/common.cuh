@@ -347,6 +347,16 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// 32-byte global store (sm_100): 16 bf16 values packed from v[0..16); p must be
+// 32-byte aligned.  One store covers a whole 32-byte sector.
+__device__ __forceinline__ void st_global_bf16x16(void* p, const float* v) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(pack_bf16x2(v[0], v[1])),
+               "r"(pack_bf16x2(v[2], v[3])), "r"(pack_bf16x2(v[4], v[5])), "r"(pack_bf16x2(v[6], v[7])),
+               "r"(pack_bf16x2(v[8], v[9])), "r"(pack_bf16x2(v[10], v[11])), "r"(pack_bf16x2(v[12], v[13])),
+               "r"(pack_bf16x2(v[14], v[15]))
+               : "memory");
+}
+
 template <typename T>
 struct Elem;
 template <>

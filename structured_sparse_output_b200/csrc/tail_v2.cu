@@ -48,6 +48,7 @@ struct StepArgs {
   const int32_t* pos_ptr;
   const int32_t* pos_ids;
   float grad_scale;
+  int dw_v8;  // dW is 32-byte aligned: the readout may use 32-byte stores
 };
 
 // Rows of the weight-stationary MMAs for groups of G labels.
@@ -631,7 +632,19 @@ __global__ void __launch_bounds__(step_threads(step_wide(kG, kUpd)), 1)
         else tmem_ld16(D(s) + lane_off + (uint32_t)(hh * NSL + c), *reinterpret_cast<float(*)[16]>(&v[c]));
       }
       tmem_wait_ld();
-      if (mvalid) {
+      bool stored = false;
+      if constexpr (kUpd == 0 && NSL % 16 == 0) {
+        // a thread's run is one label row of NSL consecutive slots, 32-byte aligned
+        // when dW is: 32-byte stores, one sector each
+        if (a.dw_v8) {
+          if (mvalid) {
+#pragma unroll
+            for (int c = 0; c < NSL / 16; ++c) st_global_bf16x16(a.dW + o + 16 * c, &v[16 * c]);
+          }
+          stored = true;
+        }
+      }
+      if (!stored && mvalid) {
 #pragma unroll
         for (int c = 0; c < NSL / 8; ++c) {
           float d8[8];
