@@ -22,8 +22,8 @@
 //              positives of the group come from a per-row cursor over the sorted
 //              CSR targets, turned into label x row bit masks in shared memory.
 //              The BCE of group i+1 comes before the dW readout of group i, so the
-//              dW product runs behind it.  The readout writes dW as 16-byte
-//              vectors (one label row, consecutive slots), or (kUpd > 0) applies an
+//              dW product runs behind it.  The readout writes dW as 32-byte
+//              (or 16-byte) vectors of one label row, or (kUpd > 0) applies an
 //              SGD update to the group's weights while dW is on chip:
 //              M' = momentum * M + dW (kUpd = 2) or M' = dW (kUpd = 1),
 //              W' = W - lr * M', with W' written to a separate buffer (the dX pass
