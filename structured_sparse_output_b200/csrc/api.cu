@@ -833,7 +833,8 @@ haste_status_t bce_step_impl(haste_plan_t p, int32_t B, haste_dtype_t dt, const 
       sa.sh = a.sh;
       sa.idx = p->idx_d;
       sa.dW = static_cast<__nv_bfloat16*>(dW);
-      sa.dw_v8 = (reinterpret_cast<uintptr_t>(dW) & 31) == 0;
+      auto a32 = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 31) == 0; };
+      sa.out_v8 = a32(dW);
       sa.dY_out = static_cast<__nv_bfloat16*>(a.dY_out);
       sa.loss_part = a.loss_part;
       sa.pos_ptr = pos.row_ptr;
@@ -846,6 +847,7 @@ haste_status_t bce_step_impl(haste_plan_t p, int32_t B, haste_dtype_t dt, const 
         sa.lr = upd->lr;
         sa.momentum = upd->momentum;
         mode = upd->momentum != 0.f ? 2 : 1;
+        sa.out_v8 = a32(upd->W_out) && (mode == 1 || a32(upd->M));
       }
       e = tail2::launch_step(p->G, p->k, mode, sa, grid, a.Xt, W, s);
     } else {

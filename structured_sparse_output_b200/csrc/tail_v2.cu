@@ -48,7 +48,7 @@ struct StepArgs {
   const int32_t* pos_ptr;
   const int32_t* pos_ids;
   float grad_scale;
-  int dw_v8;  // dW is 32-byte aligned: the readout may use 32-byte stores
+  int out_v8;  // the readout's outputs (dW, or W_out and M) are 32-byte aligned: 32-byte stores
 };
 
 // Rows of the weight-stationary MMAs for groups of G labels.
@@ -633,13 +633,32 @@ __global__ void __launch_bounds__(step_threads(step_wide(kG, kUpd)), 1)
       }
       tmem_wait_ld();
       bool stored = false;
-      if constexpr (kUpd == 0 && NSL % 16 == 0) {
+      if constexpr (NSL % 16 == 0) {
         // a thread's run is one label row of NSL consecutive slots, 32-byte aligned
-        // when dW is: 32-byte stores, one sector each
-        if (a.dw_v8) {
+        // when the outputs are: 32-byte stores, one sector each
+        if (a.out_v8) {
           if (mvalid) {
 #pragma unroll
-            for (int c = 0; c < NSL / 16; ++c) st_global_bf16x16(a.dW + o + 16 * c, &v[16 * c]);
+            for (int c2 = 0; c2 < NSL / 16; ++c2) {
+              if constexpr (kUpd == 0) {
+                st_global_bf16x16(a.dW + o + 16 * c2, &v[16 * c2]);
+              } else {
+                float mo[16], wo[16];
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                  const __nv_bfloat16* wb = reinterpret_cast<const __nv_bfloat16*>(&wv[2 * c2 + h]);
+                  const __nv_bfloat16* mb = reinterpret_cast<const __nv_bfloat16*>(&mv[2 * c2 + h]);
+#pragma unroll
+                  for (int e = 0; e < 8; ++e) {
+                    const float d = v[16 * c2 + 8 * h + e];
+                    mo[8 * h + e] = kUpd == 2 ? fmaf(a.momentum, __bfloat162float(mb[e]), d) : d;
+                    wo[8 * h + e] = fmaf(-a.lr, mo[8 * h + e], __bfloat162float(wb[e]));
+                  }
+                }
+                if constexpr (kUpd == 2) st_global_bf16x16(a.M + o + 16 * c2, mo);
+                st_global_bf16x16(a.W_out + o + 16 * c2, wo);
+              }
+            }
           }
           stored = true;
         }
