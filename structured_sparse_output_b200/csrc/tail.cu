@@ -158,7 +158,7 @@ __device__ __forceinline__ void issue_z(uint32_t d_tmem, uint32_t dy, uint32_t w
 }
 
 // Bounded wait of the whole block on an MMA-completion barrier; returns false on
-// timeout (every thread sees the same verdict).
+// timeout (every thread sees the same outcome).
 __device__ __forceinline__ bool block_wait(uint64_t* bar, uint32_t& phase, int* abort_flag) {
   const bool ok = mbar_wait(bar, phase);
   phase ^= 1u;
